@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of one PagedAttention decode step on B200.
+
+A step is the whole hot path over one batch: the cache append
+(pa_reshape_and_cache) followed by paged decode attention (pa_decode: the
+split-context kernel plus its log-sum-exp merge).  Default workload: the
+LLaMA-7B-shaped layer (32 sequences, 32 q / 32 kv heads, head_dim 128,
+block_size 16, context lengths uniform in [128, 2048], fp16, a shuffled pool
+of 8400 blocks).
+
+Metric: effective HBM bandwidth = logical K+V bytes the step reads
+(sum over sequences of ctx * kv_heads * head_dim * 2 * 2 B) / device time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent
+replica of the workload (decode shards over sequences with no exchange);
+`value` is the bytes of all ranks / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "pa_decode effective HBM GB/s (KV bytes read / device time) and % of B200 peak"
+UNIT = "GB/s"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+# DRAM traffic of one decode launch (dram__bytes_read.sum + dram__bytes_write.sum
+# from an ncu capture), keyed by workload, valid only while the kernel sources
+# hash to `src`.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("paged_decode.cu", "pa_device.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_368_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def describe(wl) -> str:
+    ctx = wl.context_lens
+    return (f"{wl.name}: {wl.num_seqs} seqs, {wl.num_heads} q / {wl.num_kv_heads} kv heads, head_dim "
+            f"{wl.head_dim}, block_size {wl.block_size}, ctx {int(ctx.min())}..{int(ctx.max())} "
+            f"(mean {float(ctx.mean()):.0f}), {wl.dtype}, pool {wl.num_blocks} blocks shuffled")
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[0]), float(parts[1]), parts[2], parts[3:7]))
+            except ValueError:
+                continue
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside if inside else self.samples
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({names[i] for s in use for i, v in enumerate(s[4]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": max(s[2] for s in use),
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# ------------------------------------------------------------------ distributed
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def load_workload(args, poison=False):
+    from paged_kv_cache_368_b200 import inputs
+
+    return inputs.config(args.config, block_size=args.block_size, poison=poison)
+
+
+# ------------------------------------------------------------------ oracle timing (CPU)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_pass(wl, units):
+    """Prepare the float64 oracle (append + decode) on `units` = [(seq, kv_head)]
+    of the workload.  Returns (run, kv_bytes): run() does one pass."""
+    import oracle
+
+    G = wl.num_heads // wl.num_kv_heads
+    seqs = sorted({s for s, _ in units})
+    kc, vc, tc = wl.compact(seqs)
+    row = {s: r for r, s in enumerate(seqs)}
+    slots = np.array([oracle.slot_of_position(tc[row[s]], int(wl.context_lens[s]) - 1, wl.block_size)
+                      for s in seqs], dtype=np.int64)
+    by_head = {}
+    for s, h in units:
+        by_head.setdefault(h, []).append(s)
+    nbytes = sum(int(wl.context_lens[s]) for s, _ in units) * wl.head_dim * 2 * wl.elem_bytes
+
+    def run():
+        k2, v2 = oracle.reshape_and_cache(wl.k_new[seqs], wl.v_new[seqs], kc, vc, slots)
+        for h, ss in by_head.items():
+            rows = [row[s] for s in ss]
+            oracle.decode(wl.q[ss][:, h * G:(h + 1) * G], k2[:, h:h + 1], v2[:, h:h + 1], tc[rows],
+                          wl.context_lens[ss], wl.scale, wl.dtype)
+
+    return run, nbytes
+
+
+def time_passes(run, budget_s):
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while True:
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() > t_end:
+            break
+    return statistics.median(times), len(times)
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    # bound the sample: time one sequence, then take as many whole sequences as fit
+    run1, _ = oracle_pass(wl, [(0, h) for h in range(wl.num_kv_heads)])
+    per_seq, _ = time_passes(run1, 0.0)
+    nseq = int(max(1, min(wl.num_seqs, budget_s / 3 / max(per_seq, 1e-4))))
+    run, nbytes = oracle_pass(wl, [(s, h) for s in range(nseq) for h in range(wl.num_kv_heads)])
+    t, reps = time_passes(run, budget_s)
+    return {"value": nbytes / t / 1e9, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"float64 NumPy oracle (append + decode) on sequences 0..{nseq - 1} of {wl.num_seqs}, "
+                       f"all {wl.num_kv_heads} kv-heads ({nbytes / 1e6:.1f} MB KV), median of {reps} passes"),
+            "host_cpus": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args):
+    world, rank, _ = dist_init()
+    if rank != 0:
+        return 0
+    wl = load_workload(args)
+    K, W = args.steps, args.warmup
+    units = [(s, h) for s in range(wl.num_seqs) for h in range(wl.num_kv_heads)]
+    run1, _ = oracle_pass(wl, units[:1])
+    t1, _ = time_passes(run1, 0.0)
+    budget = 120.0  # seconds for the whole warm-up + timed run
+    n_units = int(max(1, min(len(units), budget / max(K + W, 1) / max(t1, 1e-5))))
+    run, nbytes = oracle_pass(wl, units[:n_units])
+    for _ in range(W):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        run()
+    total = time.perf_counter() - t0
+    value = nbytes * K / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": total / K * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(wl), "sample_units": n_units, "parallelism": "none (CPU, rank 0)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{n_units} (sequence, kv-head) units per step of {len(units)}, "
+                                   f"{nbytes / 1e6:.2f} MB KV per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+
+def run_ours(args):
+    import ctypes
+
+    import torch
+
+    from paged_kv_cache_368_b200 import build as pbuild
+    from paged_kv_cache_368_b200 import libpaged
+
+    world, rank, local = dist_init()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if rank == 0:
+        pbuild.build()
+    if dist is not None:
+        dist.barrier()
+    lib = libpaged.load()
+
+    wl = load_workload(args)
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+    dev = torch.device("cuda", local)
+
+    def upload(raw):
+        return torch.from_numpy(np.ascontiguousarray(raw).view(np.int16).copy()).view(dt).to(dev)
+
+    shape = (wl.num_blocks, wl.num_kv_heads, wl.block_size, wl.head_dim)
+    k_cache = torch.zeros(shape, dtype=dt, device=dev)
+    v_cache = torch.zeros(shape, dtype=dt, device=dev)
+    idx = torch.from_numpy(wl.used).to(dev)
+    k_cache.index_copy_(0, idx, upload(wl.k_blocks))
+    v_cache.index_copy_(0, idx, upload(wl.v_blocks))
+    q, k_new, v_new = upload(wl.q), upload(wl.k_new), upload(wl.v_new)
+    slots = torch.from_numpy(wl.slot_mapping.astype(np.int64)).to(dev)
+    tables = torch.from_numpy(wl.block_tables.astype(np.int32)).to(dev)
+    ctx = torch.from_numpy(wl.context_lens.astype(np.int32)).to(dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    max_ctx = wl.max_context_len
+    ws = libpaged.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, max_ctx, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    kvh, D, bs, nb = wl.num_kv_heads, wl.head_dim, wl.block_size, wl.num_blocks
+    code = libpaged.dtype_code(dt)
+    mb = wl.max_blocks_per_seq
+    r_args = (k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), slots.data_ptr(),
+              wl.num_seqs, kvh, D, bs, nb, code, err.data_ptr(), sp)
+    d_args = (out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), tables.data_ptr(), mb,
+              ctx.data_ptr(), wl.num_seqs, max_ctx, float(wl.scale), wl.num_heads, kvh, D, bs, nb, code,
+              ws.data_ptr(), ws.numel(), 0, err.data_ptr(), sp)
+
+    def step(dec_events=None):
+        st = lib.pa_reshape_and_cache(*r_args)
+        if dec_events is not None:
+            dec_events[0].record(stream)
+        st |= lib.pa_decode(*d_args)
+        if dec_events is not None:
+            dec_events[1].record(stream)
+        return st
+
+    K, W = args.steps, args.warmup
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
+    time.sleep(0.3)
+    for _ in range(W):
+        if step() != 0:
+            raise SystemExit("libpaged call failed in warm-up")
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error flags {int(err.item())}")
+
+    dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    e0.record(stream)
+    bad = 0
+    for i in range(K):
+        bad |= step(dec[i])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if dist is not None:
+        dist.barrier()
+    if bad:
+        raise SystemExit("libpaged call failed in the timed region")
+    elapsed_ms = e0.elapsed_time(e1)
+    dec_ms = [a.elapsed_time(b) for a, b in dec]
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # ---- end to end through the public API: host buffers in, result out
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+    h_q = pin(wl.q.view(np.int16)).view(dt)
+    h_k, h_v = pin(wl.k_new.view(np.int16)).view(dt), pin(wl.v_new.view(np.int16)).view(dt)
+    h_slots = pin(wl.slot_mapping.astype(np.int64))
+    h_tables = pin(wl.block_tables.astype(np.int32))
+    h_ctx = pin(wl.context_lens.astype(np.int32))
+    h_out = torch.empty(out.shape, dtype=dt).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_ctx))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        k_new.copy_(h_k, non_blocking=True)
+        v_new.copy_(h_v, non_blocking=True)
+        slots.copy_(h_slots, non_blocking=True)
+        tables.copy_(h_tables, non_blocking=True)
+        ctx.copy_(h_ctx, non_blocking=True)
+        libpaged.reshape_and_cache(k_new, v_new, k_cache, v_cache, slots, err_flags=err)
+        libpaged.decode(out, q, k_cache, v_cache, tables, ctx, float(wl.scale), max_context_len=max_ctx,
+                        workspace=ws, err_flags=err)
+        h_out.copy_(out, non_blocking=True)
+
+    Ke = min(K, 2000)
+    for _ in range(max(3, W)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    clocks.stop()
+
+    kvb = wl.kv_bytes()
+    value = kvb * world * K / (elapsed_ms * 1e-3) / 1e9
+    mean_dec = statistics.mean(dec_ms)
+    achieved = kvb / (mean_dec * 1e-3) / 1e9
+    peak, peak_src = measured_peak()
+    src = kernel_source_hash()
+    tr = NCU_TRAFFIC.get(wl.name)
+    traffic = tr["bytes"] if tr and tr.get("src") == src else None
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(load_workload(args))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": describe(wl), "kv_bytes_per_step": kvb, "unique_kv_bytes_per_step": wl.unique_kv_bytes(),
+                   "l2": f"inputs larger than L2 ({kvb / 2**20:.0f} MiB of KV per step vs 126 MiB L2); no flush",
+                   "parallelism": f"{world} independent replica(s), one per GPU", "step": "append + decode + merge"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "kernel": "pa_decode (decode + merge launches)",
+                     "peak_source": peak_src, "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,
+                     "decode_us_mean": mean_dec * 1e3, "decode_us_median": statistics.median(dec_ms) * 1e3,
+                     "decode_us_min": min(dec_ms) * 1e3, "kernel_src": src},
+        "cpu_baseline": cpu,
+        "e2e": {"value": kvb * Ke / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke, "ms_per_step": e2e_ms / Ke,
+                "path": "pinned host -> device copies, libpaged.reshape_and_cache + libpaged.decode, device -> pinned host"},
+        "gpu_launches": 3 * K,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, default=1, help="workload index (1 = LLaMA-7B-shaped layer)")
+    ap.add_argument("--block-size", type=int, default=None, help="block size for workload 3 (LLaMA-13B)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

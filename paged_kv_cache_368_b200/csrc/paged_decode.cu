@@ -1,0 +1,913 @@
+// Paged decode attention for B200 (sm_100a).
+//
+// What is computed ("【infra之路】10-PagedAttention 与 KV Cache 管理"):
+//   section 1.1 -- one new query per sequence attends over every cached token,
+//                  out = softmax(q K^T * scale) V;
+//   sections 3.2-3.4 -- K/V live in fixed-size physical blocks reached through a
+//                  per-sequence block table; attention itself is unchanged;
+//   section 8 (Q2, Q3) -- long contexts are split FlashDecoding-style and the
+//                  pieces are combined; the kernel tiles like FlashAttention
+//                  (running max / running sum, "online softmax").
+//
+// Design (B200-first; the pages' own Ascend kernel copies scattered pages into
+// a contiguous buffer first, which this design does not do):
+//  * Work unit = (sequence, kv-head).  Its context is cut into chunks of 16
+//    tokens.  All chunks of all units are laid end to end (sequence-major,
+//    then kv-head, then chunk) and split evenly over every warp of a
+//    persistent grid (one CTA per SM, 8 warps each): each warp owns one
+//    contiguous run of chunks, so mixed context lengths balance to within a
+//    chunk and no partition-size heuristic is needed.
+//  * A warp's run is cut at unit boundaries into segments.  A segment that
+//    covers a whole unit writes the normalised output directly; a unit split
+//    across warps leaves un-normalised partials (m, l, o) that the merge
+//    kernel combines by log-sum-exp.
+//  * Each warp is its own producer: lane 0 issues TMA tile loads (128-byte
+//    swizzle, L2 evict-first) of the K and V rows of chunk k+DEPTH into a
+//    per-warp ring of shared-memory stages, completion counted on an
+//    mbarrier, while the warp computes on chunk k.  Block-table entries for
+//    the next 32 chunks are fetched with one coalesced load (one per lane)
+//    and kept in registers.
+//  * Groups of 1-2 q-heads per kv-head (MHA) use CUDA cores: 16 lanes cover
+//    one 256-byte K row (one 16-byte vector each), partial dot products of
+//    8 tokens are reduced with a transposing shuffle tree.  Groups of 4-8
+//    q-heads (GQA) form a real contraction: S = Q K^T and O += P V run on
+//    the tensor cores (mma.sync m16n8k16, q-heads on M), fed by ldmatrix
+//    from the swizzled tiles.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <mutex>
+#include <type_traits>
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+constexpr int kChunk = 16;       // tokens per pipeline stage
+constexpr int kMaxSeqs = 2048;   // prefix table lives in shared memory
+constexpr int kWarps = 8;        // warps per CTA
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+struct DecodeParams {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* ws_o;       // [2W][G][D] un-normalised partial outputs
+  float2* ws_ml;     // [2W][G] (running max in log2 units, running sum)
+  int4* ws_jobs;     // [W] merge jobs
+  int* ws_header;    // [0] = total chunks
+  int32_t* err_flags;
+  int64_t num_blocks;
+  int num_seqs;
+  int max_blocks_per_seq;
+  int ctx_cap;       // min(max_context_len, max_blocks_per_seq * block_size)
+  int max_context_len;
+  int num_heads;
+  int num_kv_heads;
+  int block_size;
+  int total_warps;
+  float scale_log2;  // scale * log2(e)
+};
+
+template <int D, int G>
+struct Shape {
+  static constexpr bool kMma = G >= 4;
+  static constexpr int kDepth = D == 64 ? 4 : (kMma ? 2 : 3);
+  static constexpr int kTileBytes = kChunk * D * 2;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kQBytes = G * D * 2;
+  static constexpr int kStages = kWarps * kDepth;
+  static constexpr size_t kFixedSmem =
+      1024 + size_t(kStages) * kStageBytes + size_t(kStages) * kQBytes + size_t(kStages) * 8;
+  static size_t smem_bytes(int num_seqs) { return kFixedSmem + ((size_t(num_seqs) + 1) * 4 + 15) / 16 * 16; }
+};
+
+// --------------------------------------------------------------- chunk lookup
+
+struct ChunkInfo {
+  int seq;    // -1: no chunk
+  int head;   // kv-head
+  int c;      // chunk index inside the unit
+  int nc;     // chunks in the unit
+  int p0;     // physical block of the chunk's first rows
+  int p1;     // second physical block (block_size 8), or -1
+  int valid;  // tokens of the chunk inside the context; 0 = skip the chunk
+  int row0;   // first row of the chunk inside block p0
+};
+
+__device__ __forceinline__ int clamp_ctx(int ctx, int cap) { return ctx < 0 ? 0 : (ctx > cap ? cap : ctx); }
+
+// Chunk `g` of the global chunk order (g < total).  `prefix[s]` = chunks of
+// sequences < s, per kv-head.
+__device__ __forceinline__ ChunkInfo chunk_info(const DecodeParams& p, const int* prefix, int64_t g, int64_t end) {
+  ChunkInfo ci;
+  ci.seq = -1;
+  ci.head = ci.c = ci.nc = ci.p0 = ci.row0 = 0;
+  ci.p1 = -1;
+  ci.valid = 0;
+  if (g >= end) return ci;
+  const int KVH = p.num_kv_heads;
+  int lo = 0, hi = p.num_seqs;  // largest s in [0, S) with KVH*prefix[s] <= g
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)KVH * prefix[mid] <= g) lo = mid; else hi = mid;
+  }
+  const int s = lo;
+  const int nc = prefix[s + 1] - prefix[s];
+  const int rem = static_cast<int>(g - (int64_t)KVH * prefix[s]);
+  const int h = rem / nc;
+  const int c = rem - h * nc;
+  const int ctx = clamp_ctx(__ldg(p.context_lens + s), p.ctx_cap);
+  const int t0 = c * kChunk;
+  const int bs = p.block_size;
+  const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+  int p0, p1 = -1, row0 = 0;
+  if (bs >= kChunk) {
+    p0 = __ldg(row + t0 / bs);
+    row0 = t0 % bs;
+  } else {  // two blocks of 8 tokens
+    p0 = __ldg(row + 2 * c);
+    if (t0 + 8 < ctx) p1 = __ldg(row + 2 * c + 1);
+  }
+  bool ok = p0 >= 0 && p0 < p.num_blocks;
+  if (p1 != -1) ok = ok && p1 >= 0 && p1 < p.num_blocks;
+  if (!ok) set_err(p.err_flags, PA_ERRF_BLOCK_RANGE);
+  ci.seq = s;
+  ci.head = h;
+  ci.c = c;
+  ci.nc = nc;
+  ci.p0 = p0;
+  ci.p1 = ok ? p1 : -1;
+  ci.valid = ok ? min(kChunk, ctx - t0) : 0;
+  ci.row0 = row0;
+  return ci;
+}
+
+__device__ __forceinline__ ChunkInfo shfl_info(const ChunkInfo& a, int src) {
+  ChunkInfo r;
+  r.seq = __shfl_sync(kFull, a.seq, src);
+  r.head = __shfl_sync(kFull, a.head, src);
+  r.c = __shfl_sync(kFull, a.c, src);
+  r.nc = __shfl_sync(kFull, a.nc, src);
+  r.p0 = __shfl_sync(kFull, a.p0, src);
+  r.p1 = __shfl_sync(kFull, a.p1, src);
+  r.valid = __shfl_sync(kFull, a.valid, src);
+  r.row0 = __shfl_sync(kFull, a.row0, src);
+  return r;
+}
+
+// --------------------------------------------------------------- CUDA-core path
+
+template <typename T, int D, int G>
+struct CoreWarp {
+  using E = Elem<T>;
+  static constexpr int LPT = D / 8;         // lanes per 16-byte-vectorised row
+  static constexpr int TPW = 32 / LPT;      // token rows per warp instruction
+  static constexpr int IT = kChunk / TPW;   // instructions per chunk
+
+  float qf[G][8];
+  float o[G][8];
+  float m[G], l[G];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
+    }
+  }
+
+  __device__ __forceinline__ void load_q(uint32_t qslot, float scale_log2, int lane) {
+    const int j = lane % LPT;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const uint4 u = lds128(qslot + g * D * 2 + j * 16);
+      const float2 a = E::to_f2(u.x), b = E::to_f2(u.y), c = E::to_f2(u.z), d = E::to_f2(u.w);
+      qf[g][0] = a.x * scale_log2; qf[g][1] = a.y * scale_log2;
+      qf[g][2] = b.x * scale_log2; qf[g][3] = b.y * scale_log2;
+      qf[g][4] = c.x * scale_log2; qf[g][5] = c.y * scale_log2;
+      qf[g][6] = d.x * scale_log2; qf[g][7] = d.y * scale_log2;
+    }
+  }
+
+  template <bool kMasked>
+  __device__ __forceinline__ void chunk(uint32_t ktile, uint32_t vtile, int valid, int lane) {
+    const int grp = lane / LPT, j = lane % LPT;
+    float acc[G][IT];
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int tok = it * TPW + grp;
+      const uint4 u = lds128(ktile + tile_off(tok, j));
+      const float2 a = E::to_f2(u.x), b = E::to_f2(u.y), c = E::to_f2(u.z), d = E::to_f2(u.w);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float s = qf[g][0] * a.x;
+        s = fmaf(qf[g][1], a.y, s);
+        s = fmaf(qf[g][2], b.x, s);
+        s = fmaf(qf[g][3], b.y, s);
+        s = fmaf(qf[g][4], c.x, s);
+        s = fmaf(qf[g][5], c.y, s);
+        s = fmaf(qf[g][6], d.x, s);
+        s = fmaf(qf[g][7], d.y, s);
+        acc[g][it] = s;
+      }
+    }
+    // Transposing reduction over the LPT lanes of a row group: each step
+    // halves the values a lane keeps; afterwards lane j holds the full dot
+    // product of token (j >> 1) * TPW + grp (lanes j and j^1 agree).
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int step = IT / 2, mask = LPT / 2; step >= 1; step >>= 1, mask >>= 1) {
+        const bool upper = (j & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < step; ++i) {
+          const float send = upper ? acc[g][i] : acc[g][i + step];
+          const float keep = upper ? acc[g][i + step] : acc[g][i];
+          acc[g][i] = keep + __shfl_xor_sync(kFull, send, mask);
+        }
+      }
+      acc[g][0] += __shfl_xor_sync(kFull, acc[g][0], 1);
+    }
+    const int my_tok = (j >> 1) * TPW + grp;
+    float pg[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float s = (!kMasked || my_tok < valid) ? acc[g][0] : -INFINITY;
+      float cm = s;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, off));
+      const float mn = fmaxf(m[g], cm);
+      const float alpha = fast_exp2(m[g] - mn);
+      const float pv = fast_exp2(s - mn);
+      l[g] = l[g] * alpha + ((j & 1) ? 0.f : pv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[g][e] *= alpha;
+      m[g] = mn;
+      pg[g] = pv;
+    }
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int tok = it * TPW + grp;
+      float pt[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) pt[g] = __shfl_sync(kFull, pg[g], grp * LPT + 2 * it);
+      if (!kMasked || tok < valid) {
+        const uint4 u = lds128(vtile + tile_off(tok, j));
+        const float2 a = E::to_f2(u.x), b = E::to_f2(u.y), c = E::to_f2(u.z), d = E::to_f2(u.w);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          o[g][0] = fmaf(pt[g], a.x, o[g][0]);
+          o[g][1] = fmaf(pt[g], a.y, o[g][1]);
+          o[g][2] = fmaf(pt[g], b.x, o[g][2]);
+          o[g][3] = fmaf(pt[g], b.y, o[g][3]);
+          o[g][4] = fmaf(pt[g], c.x, o[g][4]);
+          o[g][5] = fmaf(pt[g], c.y, o[g][5]);
+          o[g][6] = fmaf(pt[g], d.x, o[g][6]);
+          o[g][7] = fmaf(pt[g], d.y, o[g][7]);
+        }
+      }
+    }
+  }
+
+  // Sum the row groups and the lanes' running sums.
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int off = LPT; off < 32; off <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[g][e] += __shfl_xor_sync(kFull, o[g][e], off);
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) l[g] += __shfl_xor_sync(kFull, l[g], off);
+    }
+  }
+
+  __device__ __forceinline__ void write_out(T* out_row, int lane) const {  // out_row -> [G][D]
+    const int j = lane % LPT;
+    if (lane >= LPT) return;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float inv = l[g] > 0.f ? 1.f / l[g] : 0.f;
+      uint4 u;
+      u.x = E::pack(o[g][0] * inv, o[g][1] * inv);
+      u.y = E::pack(o[g][2] * inv, o[g][3] * inv);
+      u.z = E::pack(o[g][4] * inv, o[g][5] * inv);
+      u.w = E::pack(o[g][6] * inv, o[g][7] * inv);
+      *reinterpret_cast<uint4*>(out_row + g * D + j * 8) = u;
+    }
+  }
+
+  __device__ __forceinline__ void write_partial(float* po, float2* pml, int lane) const {  // po -> [G][D]
+    const int j = lane % LPT;
+    if (lane < LPT) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float4* dst = reinterpret_cast<float4*>(po + g * D + j * 8);
+        dst[0] = make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+        dst[1] = make_float4(o[g][4], o[g][5], o[g][6], o[g][7]);
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) pml[g] = make_float2(m[g], l[g]);
+    }
+  }
+};
+
+// --------------------------------------------------------------- tensor-core path
+
+template <typename T, int D, int G>
+struct MmaWarp {
+  using E = Elem<T>;
+  static constexpr int NT = D / 8;   // 8-wide output column tiles
+  static constexpr int KS = D / 16;  // k-steps of the QK product
+
+  uint32_t qa[KS][2];  // A fragments of Q (rows = q-heads 0..7; rows 8..15 are zero)
+  float o[NT][2];      // O rows gid, columns 8*n + 2*tq + {0,1}
+  float m, l;
+
+  // D[0..1] += A * B for the upper 8 rows of a 16x8 tile; the lower rows of A
+  // are zero, so the lower rows of D are discarded.
+  __device__ static __forceinline__ void mma_top(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
+                                                 uint32_t b1) {
+    float d[4] = {d0, d1, 0.f, 0.f};
+    E::mma(d, a0, 0u, a2, 0u, b0, b1);
+    d0 = d[0];
+    d1 = d[1];
+  }
+
+  __device__ __forceinline__ void reset() {
+    m = -INFINITY;
+    l = 0.f;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = 0.f;
+  }
+
+  __device__ __forceinline__ void load_q(uint32_t qslot, float /*scale_log2*/, int lane) {
+    const int gid = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a0 = 0u, a2 = 0u;
+      if (gid < G) {
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(qslot + (gid * D + ks * 16 + 2 * tq) * 2));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(qslot + (gid * D + ks * 16 + 8 + 2 * tq) * 2));
+      }
+      qa[ks][0] = a0;
+      qa[ks][1] = a2;
+    }
+  }
+
+  template <bool kMasked>
+  __device__ __forceinline__ void chunk(uint32_t ktile, uint32_t vtile, int valid, int lane, float scale_log2) {
+    const int gid = lane >> 2, tq = lane & 3;
+    // S = Q K^T for tokens 0-7 (n-tile 0) and 8-15 (n-tile 1); two
+    // accumulators per tile (even/odd k-step pairs) shorten the mma chains.
+    float s[2][2][2] = {};
+#pragma unroll
+    for (int kp = 0; kp < D / 32; ++kp) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(ktile + tile_off(nt * 8 + (lane & 7), kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_top(s[nt][kp & 1][0], s[nt][kp & 1][1], qa[2 * kp][0], qa[2 * kp][1], b0, b1);
+        mma_top(s[nt][kp & 1][0], s[nt][kp & 1][1], qa[2 * kp + 1][0], qa[2 * kp + 1][1], b2, b3);
+      }
+    }
+    float sc[4];
+    sc[0] = (s[0][0][0] + s[0][1][0]) * scale_log2;
+    sc[1] = (s[0][0][1] + s[0][1][1]) * scale_log2;
+    sc[2] = (s[1][0][0] + s[1][1][0]) * scale_log2;
+    sc[3] = (s[1][0][1] + s[1][1][1]) * scale_log2;
+    if (kMasked) {
+      const int t0 = 2 * tq;
+      if (t0 >= valid) sc[0] = -INFINITY;
+      if (t0 + 1 >= valid) sc[1] = -INFINITY;
+      if (t0 + 8 >= valid) sc[2] = -INFINITY;
+      if (t0 + 9 >= valid) sc[3] = -INFINITY;
+    }
+    float cm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
+    cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
+    const float mn = fmaxf(m, cm);
+    const float alpha = fast_exp2(m - mn);
+    float pr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[i] = fast_exp2(sc[i] - mn);
+    l = l * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+    m = mn;
+    if (!__all_sync(kFull, alpha == 1.f)) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] *= alpha;
+        o[n][1] *= alpha;
+      }
+    }
+    uint32_t a0 = E::pack(pr[0], pr[1]);
+    uint32_t a2 = E::pack(pr[2], pr[3]);
+    if (gid >= G) a0 = a2 = 0u;
+    // O += P V: B fragments of V (k = tokens, n = 8 output columns) by ldmatrix.trans.
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(vtile + tile_off(((lane >> 3) & 1) * 8 + (lane & 7), 2 * np + (lane >> 4)), b0, b1, b2,
+                        b3);
+      mma_top(o[2 * np][0], o[2 * np][1], a0, a2, b0, b1);
+      mma_top(o[2 * np + 1][0], o[2 * np + 1][1], a0, a2, b2, b3);
+    }
+  }
+
+  __device__ __forceinline__ void finish() {
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+  }
+
+  __device__ __forceinline__ void write_out(T* out_row, int lane) const {  // out_row -> [G][D]
+    const int gid = lane >> 2, tq = lane & 3;
+    if (gid >= G) return;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      *reinterpret_cast<uint32_t*>(out_row + gid * D + n * 8 + 2 * tq) = E::pack(o[n][0] * inv, o[n][1] * inv);
+  }
+
+  __device__ __forceinline__ void write_partial(float* po, float2* pml, int lane) const {
+    const int gid = lane >> 2, tq = lane & 3;
+    if (gid >= G) return;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      *reinterpret_cast<float2*>(po + gid * D + n * 8 + 2 * tq) = make_float2(o[n][0], o[n][1]);
+    if (tq == 0) pml[gid] = make_float2(m, l);
+  }
+};
+
+// Zero V rows [valid, 16) of a chunk tile: the P V product multiplies them
+// by an exact zero weight, and 0 * NaN would poison the output.
+template <int D>
+__device__ __forceinline__ void zero_tail_rows(uint32_t vtile, int valid, int lane) {
+  const int n = (kChunk - valid) * (D / 8);
+  for (int i = lane; i < n; i += 32) {
+    const int r = valid + i / (D / 8);
+    const int c16 = i % (D / 8);
+    sts128(vtile + tile_off(r, c16), make_uint4(0u, 0u, 0u, 0u));
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+
+// --------------------------------------------------------------- prefix of chunk counts
+
+template <int NT>
+__device__ __forceinline__ void build_prefix(const DecodeParams& p, int* prefix) {
+  __shared__ int warp_tot[NT / 32];
+  const int S = p.num_seqs;
+  const int t = threadIdx.x;
+  const int per = (S + NT - 1) / NT;
+  const int s0 = min(S, t * per), s1 = min(S, s0 + per);
+  int local = 0;
+  bool bad = false;
+  for (int s = s0; s < s1; ++s) {
+    const int ctx = p.context_lens[s];
+    bad |= ctx < 0 || ctx > p.ctx_cap;
+    local += (clamp_ctx(ctx, p.ctx_cap) + kChunk - 1) / kChunk;
+  }
+  if (bad && blockIdx.x == 0) set_err(p.err_flags, PA_ERRF_CONTEXT);
+  const int lane = t & 31, warp = t >> 5;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_tot[w];
+  int run = base + incl - local;
+  for (int s = s0; s < s1; ++s) {
+    prefix[s] = run;
+    run += (clamp_ctx(p.context_lens[s], p.ctx_cap) + kChunk - 1) / kChunk;
+  }
+  if (t == NT - 1) prefix[S] = base + incl;
+}
+
+// --------------------------------------------------------------- main kernel
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kWarps * 32, 1)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                        const DecodeParams p) {
+  using SH = Shape<D, G>;
+  using Warp = typename std::conditional<SH::kMma, MmaWarp<T, D, G>, CoreWarp<T, D, G>>::type;
+  constexpr int DEPTH = SH::kDepth;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t tiles = base;
+  const uint32_t qslots = tiles + SH::kStages * SH::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SH::kStages * (SH::kStageBytes + SH::kQBytes));
+  int* prefix = reinterpret_cast<int*>(bars + SH::kStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * kWarps + warp;
+  const int W = p.total_warps;
+
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  if (lane == 0) {
+    for (int i = 0; i < DEPTH; ++i) mbar_init(&bars[warp * DEPTH + i], 1);
+    fence_barrier_init();
+  }
+  build_prefix<kWarps * 32>(p, prefix);
+  __syncthreads();
+
+  const int S = p.num_seqs, H = p.num_heads;
+  const int64_t NC = (int64_t)p.num_kv_heads * prefix[S];
+  if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_header[0] = static_cast<int>(NC);
+  const int64_t c0 = (int64_t)gw * NC / W, c1 = (int64_t)(gw + 1) * NC / W;
+  const int n = static_cast<int>(c1 - c0);
+
+  // Sequences with an empty context produce zeros.
+  for (int s = gw; s < S; s += W) {
+    if (clamp_ctx(p.context_lens[s], p.ctx_cap) == 0) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + (int64_t)s * H * D);
+      for (int i = lane; i < H * D / 8; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  const uint64_t policy = l2_evict_first_policy();
+  const int rows_per_block = p.block_size < kChunk ? p.block_size : kChunk;
+  const uint32_t box_bytes = rows_per_block * 128;
+  const T* qbase = static_cast<const T*>(p.q);
+
+  ChunkInfo cur = chunk_info(p, prefix, c0 + lane, c1);
+  ChunkInfo nxt = chunk_info(p, prefix, c0 + 32 + lane, c1);
+  int kb = 0;  // chunk index held by lane 0 of `cur`
+
+  auto get = [&](int k) -> ChunkInfo {
+    const int d = k - kb;
+    return d < 32 ? shfl_info(cur, d) : shfl_info(nxt, d - 32);
+  };
+
+  auto issue = [&](int k, const ChunkInfo& ci) {
+    if (lane != 0) return;
+    const int stage = warp * DEPTH + (k % DEPTH);
+    uint64_t* bar = &bars[stage];
+    const bool seg_start = (k == 0) || ci.c == 0;
+    const int nblk = ci.valid > 0 ? (ci.p1 >= 0 ? 2 : 1) : 0;
+    const uint32_t bytes = nblk * (D / 64) * box_bytes * 2 + (seg_start ? SH::kQBytes : 0);
+    mbar_arrive_expect_tx(bar, bytes);
+    const uint32_t kt = tiles + stage * SH::kStageBytes;
+    const uint32_t vt = kt + SH::kTileBytes;
+    for (int b = 0; b < nblk; ++b) {
+      const int phys = b == 0 ? ci.p0 : ci.p1;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const uint32_t off = c * 2048 + b * 1024;
+        tma_load_4d(kt + off, &kmap, bar, 64 * c, ci.row0, ci.head, phys, policy);
+        tma_load_4d(vt + off, &vmap, bar, 64 * c, ci.row0, ci.head, phys, policy);
+      }
+    }
+    if (seg_start) {
+      const T* src = qbase + ((int64_t)ci.seq * H + (int64_t)ci.head * G) * D;
+      bulk_load(qslots + stage * SH::kQBytes, src, SH::kQBytes, bar);
+    }
+  };
+
+  for (int i = 0; i < DEPTH && i < n; ++i) issue(i, get(i));
+
+  Warp st;
+  st.reset();
+  int seg_first_c = 0;
+  bool first_seg = true;
+  bool job_written = false;
+  bool timed_out = false;
+  int k = 0;
+  for (; k < n; ++k) {
+    if (k - kb >= 32) {
+      cur = nxt;
+      kb += 32;
+      nxt = chunk_info(p, prefix, c0 + kb + 32 + lane, c1);
+    }
+    const ChunkInfo ci = get(k);
+    const int stage = warp * DEPTH + (k % DEPTH);
+    const uint32_t parity = (k / DEPTH) & 1;
+    // Every lane waits (acquiring the TMA writes); the give-up decision is
+    // made warp-wide so that the lanes never diverge around the shuffles.
+    const bool arrived = mbar_wait_bounded(&bars[stage], parity, kWaitLimitNs);
+    if (!__all_sync(kFull, arrived)) {
+      timed_out = true;
+      break;
+    }
+    const bool seg_start = (k == 0) || ci.c == 0;
+    const bool seg_end = (k == n - 1) || ci.c == ci.nc - 1;
+    if (seg_start) {
+      st.reset();
+      st.load_q(qslots + stage * SH::kQBytes, p.scale_log2, lane);
+      seg_first_c = ci.c;
+    }
+    const uint32_t kt = tiles + stage * SH::kStageBytes;
+    const uint32_t vt = kt + SH::kTileBytes;
+    if (ci.valid == kChunk) {
+      if constexpr (SH::kMma) st.template chunk<false>(kt, vt, kChunk, lane, p.scale_log2);
+      else st.template chunk<false>(kt, vt, kChunk, lane);
+    } else if (ci.valid > 0) {
+      if constexpr (SH::kMma) {
+        zero_tail_rows<D>(vt, ci.valid, lane);
+        st.template chunk<true>(kt, vt, ci.valid, lane, p.scale_log2);
+      } else {
+        st.template chunk<true>(kt, vt, ci.valid, lane);
+      }
+    }
+    __syncwarp();
+    if (k + DEPTH < n) issue(k + DEPTH, get(k + DEPTH));
+    if (seg_end) {
+      st.finish();
+      const int kvh = ci.head;
+      if (seg_first_c == 0 && ci.c == ci.nc - 1) {
+        st.write_out(static_cast<T*>(p.out) + ((int64_t)ci.seq * H + (int64_t)kvh * G) * D, lane);
+      } else {
+        const int slot = 2 * gw + (first_seg ? 0 : 1);
+        st.write_partial(p.ws_o + (int64_t)slot * G * D, p.ws_ml + (int64_t)slot * G, lane);
+      }
+      if (k == n - 1) {
+        // The unit this warp's run ends in started here and continues in the
+        // next warps: this warp owns its merge job.
+        if (lane == 0) {
+          if (seg_first_c == 0 && ci.c < ci.nc - 1) {
+            const int64_t a = c0 + k - ci.c;
+            p.ws_jobs[gw] = make_int4(ci.seq, kvh, static_cast<int>(a), ci.nc);
+          } else {
+            p.ws_jobs[gw] = make_int4(-1, 0, 0, 0);
+          }
+        }
+        job_written = true;
+      }
+      first_seg = false;
+    }
+  }
+  if (timed_out) {
+    set_err(p.err_flags, PA_ERRF_TIMEOUT);
+    // Let this warp's copies in flight land before the CTA can exit.
+    for (int kk = k; kk < n && kk < k + DEPTH; ++kk)
+      mbar_wait_bounded(&bars[warp * DEPTH + (kk % DEPTH)], (kk / DEPTH) & 1, kWaitLimitNs);
+  }
+  if (!job_written && lane == 0) p.ws_jobs[gw] = make_int4(-1, 0, 0, 0);
+}
+
+// --------------------------------------------------------------- merge kernel
+
+// Combines the partials of every unit that was split across warps:
+//   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
+// (m in log2 units).  One warp per job.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
+  using E = Elem<T>;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int W = p.total_warps;
+  if (gw >= W) return;
+  const int4 job = p.ws_jobs[gw];
+  if (job.x < 0) return;
+  const int64_t NC = p.ws_header[0];
+  const int64_t a = job.z, b = a + job.w;
+  auto start_of = [&](int64_t w) -> int64_t { return w * NC / W; };
+  const int64_t w_last = ((b - 1 + 1) * W + NC - 1) / NC - 1;  // warp holding chunk b-1
+  constexpr int PER = D / 32;
+  for (int g = 0; g < G; ++g) {
+    float M = -INFINITY;
+    for (int64_t w = gw; w <= w_last; ++w) {
+      if (start_of(w) == start_of(w + 1)) continue;
+      const int64_t slot = 2 * w + (start_of(w) >= a ? 0 : 1);
+      M = fmaxf(M, p.ws_ml[slot * G + g].x);
+    }
+    float L = 0.f;
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+    for (int64_t w = gw; w <= w_last; ++w) {
+      if (start_of(w) == start_of(w + 1)) continue;
+      const int64_t slot = 2 * w + (start_of(w) >= a ? 0 : 1);
+      const float2 ml = p.ws_ml[slot * G + g];
+      const float e = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
+      L = fmaf(e, ml.y, L);
+      const float* po = p.ws_o + (slot * G + g) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = fmaf(e, po[i], acc[i]);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    T* dst = static_cast<T*>(p.out) + ((int64_t)job.x * p.num_heads + (int64_t)job.y * G + g) * D + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; i += 2) *reinterpret_cast<uint32_t*>(dst + i) = E::pack(acc[i] * inv, acc[i + 1] * inv);
+  }
+}
+
+}  // namespace pa
+
+// =============================================================== host side
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+
+int device_sms(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+// The (cache-pool) tensor map: dims {head_dim, block_size, kv_heads, blocks},
+// box {64 elements = 128 B, min(block_size, 16) rows, 1, 1}, 128-byte swizzle.
+bool make_cache_map(CUtensorMap* map, const void* base, int64_t nb, int kvh, int bs, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)bs, (cuuint64_t)kvh, (cuuint64_t)nb};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)bs * d * 2, (cuuint64_t)kvh * bs * d * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)(bs < 16 ? bs : 16), 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct WsLayout {
+  size_t header, jobs, ml, o, total;
+};
+
+WsLayout ws_layout(int max_warps, int G, int D) {
+  WsLayout w;
+  w.header = 0;
+  w.jobs = 256;
+  w.ml = w.jobs + (size_t(max_warps) * 16 + 255) / 256 * 256;
+  w.o = w.ml + (size_t(2) * max_warps * G * 8 + 255) / 256 * 256;
+  w.total = w.o + size_t(2) * max_warps * G * D * 4;
+  return w;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+template <typename T, int D, int G>
+pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::DecodeParams& p, int ctas,
+                        cudaStream_t stream, int dev) {
+  using SH = pa::Shape<D, G>;
+  auto kern = pa::paged_decode_kernel<T, D, G>;
+  static std::atomic<int> smem_set[kMaxDevices];
+  const size_t smem = SH::smem_bytes(p.num_seqs);
+  if (dev >= 0 && dev < kMaxDevices && smem_set[dev].load(std::memory_order_relaxed) < (int)smem) {
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if ((size_t)optin < smem) return PA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
+      return PA_ERR_CUDA;
+    smem_set[dev].store(optin, std::memory_order_relaxed);
+  }
+  kern<<<ctas, pa::kWarps * 32, smem, stream>>>(km, vm, p);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  const int merge_blocks = (p.total_warps + 7) / 8;
+  pa::paged_decode_merge_kernel<T, D, G><<<merge_blocks, 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D>
+pa_status dispatch_g(int G, const CUtensorMap& km, const CUtensorMap& vm, const pa::DecodeParams& p, int ctas,
+                     cudaStream_t s, int dev) {
+  switch (G) {
+    case 1: return launch_decode<T, D, 1>(km, vm, p, ctas, s, dev);
+    case 2: return launch_decode<T, D, 2>(km, vm, p, ctas, s, dev);
+    case 4: return launch_decode<T, D, 4>(km, vm, p, ctas, s, dev);
+    case 8: return launch_decode<T, D, 8>(km, vm, p, ctas, s, dev);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+bool valid_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
+
+}  // namespace
+
+extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                           int max_context_len) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return 0;
+  if (head_dim != 64 && head_dim != 128) return 0;
+  if (max_context_len < 0) return 0;
+  const int G = num_heads / num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const int sms = device_sms(dev);
+  if (sms <= 0) return 0;
+  return ws_layout(sms * pa::kWarps, G, head_dim).total;
+}
+
+extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                               int num_seqs, int max_context_len, float scale, int num_heads, int num_kv_heads,
+                               int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype, void* workspace,
+                               size_t workspace_bytes, int max_ctas, int32_t* err_flags, pa_stream_t stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return PA_ERR_INVALID;
+  if (max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0 || max_ctas < 0) return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID;
+  const int G = num_heads / num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!valid_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > pa::kMaxSeqs) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PA_ERR_INVALID;
+  const int64_t cap64 = std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * block_size);
+  const int ctx_cap = static_cast<int>(cap64);
+  const int64_t upper = (int64_t)num_seqs * num_kv_heads * ((cap64 + pa::kChunk - 1) / pa::kChunk);
+  if (upper >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  if (num_blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const int sms = device_sms(dev);
+  if (sms <= 0) return PA_ERR_CUDA;
+  const WsLayout L = ws_layout(sms * pa::kWarps, G, head_dim);
+  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return PA_ERR_WORKSPACE;
+
+  int ctas = static_cast<int>(std::min<int64_t>(sms, std::max<int64_t>(1, (upper + pa::kWarps * 4 - 1) / (pa::kWarps * 4))));
+  if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
+
+  CUtensorMap km, vm;
+  if (!make_cache_map(&km, k_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
+      !make_cache_map(&vm, v_cache, num_blocks, num_kv_heads, block_size, head_dim))
+    return PA_ERR_CUDA;
+
+  pa::DecodeParams p;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.ws_header = reinterpret_cast<int*>(ws + L.header);
+  p.ws_jobs = reinterpret_cast<int4*>(ws + L.jobs);
+  p.ws_ml = reinterpret_cast<float2*>(ws + L.ml);
+  p.ws_o = reinterpret_cast<float*>(ws + L.o);
+  p.err_flags = err_flags;
+  p.num_blocks = num_blocks;
+  p.num_seqs = num_seqs;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.ctx_cap = ctx_cap;
+  p.max_context_len = max_context_len;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.block_size = block_size;
+  p.total_warps = ctas * pa::kWarps;
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == PA_F16) {
+    return head_dim == 128 ? dispatch_g<__half, 128>(G, km, vm, p, ctas, s, dev)
+                           : dispatch_g<__half, 64>(G, km, vm, p, ctas, s, dev);
+  }
+  return head_dim == 128 ? dispatch_g<__nv_bfloat16, 128>(G, km, vm, p, ctas, s, dev)
+                         : dispatch_g<__nv_bfloat16, 64>(G, km, vm, p, ctas, s, dev);
+}
+
+extern "C" const char* pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID: return "PA_ERR_INVALID: invalid argument";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: shape or size outside the compiled set";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA call or kernel launch failed";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "unknown pa_status";
+}
+
+extern "C" int pa_version(void) { return 100; }

@@ -1,0 +1,166 @@
+"""Thin ctypes binding of ``libpaged.so`` (C ABI in ``include/paged.h``).
+
+Argument marshalling only: tensors are passed as raw device pointers plus
+sizes, on torch's current CUDA stream.  Every step of the computation runs in
+the library's kernels.  There is no fallback: without the built library, or
+with a tensor that is not on a CUDA device, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libpaged.so")
+
+PA_F16, PA_BF16 = 0, 1
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
+
+ERRF_SLOT_RANGE = 1 << 0
+ERRF_BLOCK_RANGE = 1 << 1
+ERRF_CONTEXT = 1 << 2
+ERRF_TIMEOUT = 1 << 3
+
+SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_status_string", "pa_version")
+
+_lib: Optional[ctypes.CDLL] = None
+
+_c = ctypes
+_vp, _i32, _i64, _f32, _sz = _c.c_void_p, _c.c_int, _c.c_int64, _c.c_float, _c.c_size_t
+
+
+class LibpagedError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load (once) and return the shared library."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError(
+            f"{p} is not built; run `python -m paged_kv_cache_368_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(p)
+    lib.pa_reshape_and_cache.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i32, _vp, _vp]
+    lib.pa_reshape_and_cache.restype = _i32
+    lib.pa_decode_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i32]
+    lib.pa_decode_workspace_size.restype = _sz
+    lib.pa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64,
+                              _i32, _vp, _sz, _i32, _vp, _vp]
+    lib.pa_decode.restype = _i32
+    lib.pa_status_string.argtypes = [_i32]
+    lib.pa_status_string.restype = _c.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = _i32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().pa_status_string(int(status)).decode()
+
+
+def dtype_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float16:
+        return PA_F16
+    if dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"libpaged supports float16 and bfloat16, not {dtype}")
+
+
+def _dev_ptr(t: Optional[torch.Tensor], name: str) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libpaged has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      slot_mapping: torch.Tensor, err_flags: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Append: ``k_cache[s // bs, :, s % bs, :] = key[n]`` for ``s = slot_mapping[n] >= 0`` (same for V).
+
+    key/value ``[T, KVH, D]``; caches ``[NB, KVH, BS, D]``; slot_mapping int64 ``[T]``."""
+    if k_cache.dim() != 4 or key.dim() != 3:
+        raise ValueError("k_cache must be [NB, KVH, BS, D] and key [T, KVH, D]")
+    nb, kvh, bs, d = k_cache.shape
+    if key.shape[1:] != (kvh, d) or value.shape != key.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between key/value and the caches")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (key.shape[0],):
+        raise ValueError("slot_mapping must be int64 [T]")
+    if not (key.dtype == value.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("key, value and caches must share one dtype")
+    st = load().pa_reshape_and_cache(
+        _dev_ptr(key, "key"), _dev_ptr(value, "value"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(slot_mapping, "slot_mapping"), key.shape[0], kvh, d, bs, nb, dtype_code(key.dtype),
+        _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_reshape_and_cache")
+
+
+def decode_workspace_size(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int,
+                          max_context_len: int) -> int:
+    return int(load().pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len))
+
+
+def alloc_workspace(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_context_len: int,
+                    device=None) -> torch.Tensor:
+    n = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len)
+    if n == 0:
+        raise LibpagedError(PA_ERR_UNSUPPORTED, "pa_decode_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device if device is not None else "cuda")
+
+
+def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+           max_context_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None, max_ctas: int = 0,
+           err_flags: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``out[s, h] = softmax(scale * q[s, h] . K_s^T) V_s`` over the paged caches.
+
+    q/out ``[S, H, D]``; caches ``[NB, KVH, BS, D]``; block_tables int32 ``[S, MB]``;
+    context_lens int32 ``[S]`` (counting the token appended this step).
+    ``max_context_len`` bounds context_lens (default ``MB * BS``, no device sync)."""
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [S, H, D] and k_cache [NB, KVH, BS, D]")
+    S, H, D = q.shape
+    nb, kvh, bs, d2 = k_cache.shape
+    if d2 != D or v_cache.shape != k_cache.shape or out.shape != q.shape:
+        raise ValueError("shape mismatch between q/out and the caches")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("block_tables must be int32 [S, MB]")
+    if context_lens.dtype != torch.int32 or context_lens.shape != (S,):
+        raise ValueError("context_lens must be int32 [S]")
+    if not (q.dtype == out.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q, out and caches must share one dtype")
+    mb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = mb * bs
+    if workspace is None:
+        workspace = alloc_workspace(S, H, kvh, D, max_context_len, device=q.device)
+    st = load().pa_decode(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(block_tables, "block_tables"), mb, _dev_ptr(context_lens, "context_lens"), S,
+        int(max_context_len), float(scale), H, kvh, D, bs, nb, dtype_code(q.dtype),
+        _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(), int(max_ctas),
+        _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_decode")
+    return out

@@ -1,0 +1,108 @@
+"""The C-ABI library loads, exports every symbol ``include/paged.h`` declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_368_b200 import build as pbuild
+from paged_kv_cache_368_b200 import libpaged
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return libpaged.load()
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert set(libpaged.SYMBOLS) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.pa_version() >= 100
+    for code in range(5):
+        assert libpaged.status_string(code).startswith("PA_")
+    assert "unknown" in libpaged.status_string(99)
+
+
+def _decode(lib, **kw):
+    a = dict(out=16, q=16, k=16, v=16, tables=16, mb=4, ctx=16, S=2, maxctx=64, scale=0.1, H=4, KVH=4, D=128,
+             BS=16, NB=8, dtype=0, ws=16, wsb=1 << 30, max_ctas=0, err=None, stream=None)
+    a.update(kw)
+    return lib.pa_decode(a["out"], a["q"], a["k"], a["v"], a["tables"], a["mb"], a["ctx"], a["S"], a["maxctx"],
+                         a["scale"], a["H"], a["KVH"], a["D"], a["BS"], a["NB"], a["dtype"], a["ws"], a["wsb"],
+                         a["max_ctas"], a["err"], a["stream"])
+
+
+def test_decode_host_checks(lib):
+    I, U = libpaged.PA_ERR_INVALID, libpaged.PA_ERR_UNSUPPORTED
+    assert _decode(lib, H=6, KVH=4) == I  # heads not a multiple of kv-heads
+    assert _decode(lib, H=0) == I
+    assert _decode(lib, S=-1) == I
+    assert _decode(lib, mb=0) == I
+    assert _decode(lib, NB=0) == I
+    assert _decode(lib, dtype=7) == I
+    assert _decode(lib, scale=float("inf")) == I
+    assert _decode(lib, max_ctas=-1) == I
+    assert _decode(lib, H=48, KVH=3) == U  # group of 16 q-heads
+    assert _decode(lib, D=96) == U
+    assert _decode(lib, BS=24) == U
+    assert _decode(lib, S=4096) == U
+    assert _decode(lib, out=None) == I
+    assert _decode(lib, q=24) == I  # misaligned
+    assert _decode(lib, S=0) == libpaged.PA_OK  # nothing to do, nothing touched
+
+
+def test_reshape_host_checks(lib):
+    f = lib.pa_reshape_and_cache
+    I, U = libpaged.PA_ERR_INVALID, libpaged.PA_ERR_UNSUPPORTED
+    ok = dict(key=16, value=16, kc=16, vc=16, slots=16, T=4, KVH=2, D=64, BS=16, NB=4, dt=0)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["key"], a["value"], a["kc"], a["vc"], a["slots"], a["T"], a["KVH"], a["D"], a["BS"], a["NB"],
+                 a["dt"], None, None)
+
+    assert call(T=-1) == I
+    assert call(KVH=0) == I
+    assert call(NB=0) == I
+    assert call(dt=5) == I
+    assert call(D=32) == U
+    assert call(BS=12) == U
+    assert call(key=None) == I
+    assert call(kc=8) == I  # misaligned
+    assert call(slots=4) == I  # misaligned int64
+    assert call(T=0) == libpaged.PA_OK
+
+
+def test_workspace_size_rejects_bad_shapes(lib):
+    assert lib.pa_decode_workspace_size(4, 6, 4, 128, 100) == 0
+    assert lib.pa_decode_workspace_size(4, 32, 2, 128, 100) == 0  # group of 16
+    assert lib.pa_decode_workspace_size(4, 8, 8, 80, 100) == 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+
+    q = torch.zeros(1, 1, 64, dtype=torch.float16)
+    kc = torch.zeros(2, 1, 16, 64, dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA"):
+        libpaged.decode(q.clone(), q, kc, kc.clone(), torch.zeros(1, 1, dtype=torch.int32),
+                        torch.ones(1, dtype=torch.int32), 0.125, workspace=torch.zeros(16, dtype=torch.uint8))

@@ -1,0 +1,274 @@
+"""GPU parity: libpaged (through its C ABI) against the float64 oracle.
+
+* append: bit-exact over the whole pool (or, for pools too big to copy
+  back, the touched rows bit-exact and every other byte unchanged);
+* decode: every output element within |gpu - ref| <= atol + rtol |ref|
+  (fp16: 2e-3 + 1e-2, bf16: 1.6e-2 + 2e-2) at small sizes; at full sizes on
+  sampled sequences and kv-heads, plus finiteness everywhere;
+* invariants that must hold bit-for-bit on the GPU: permuting physical
+  blocks, sharing prefix blocks, context length 1 returning V.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_harness import DeviceState, TOL, assert_close, reference_full, reference_sampled, to_dev, to_raw
+from paged_kv_cache_368_b200 import inputs, libpaged
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    libpaged.load()
+    yield
+
+
+# ------------------------------------------------------------------ config 0 (tiny MHA), whole thing
+
+
+def test_tiny_mha_step_matches_oracle():
+    wl = inputs.config(0)
+    ds = DeviceState(wl, full_pool=True)
+    out = ds.step()
+    ref, k_ref, v_ref = reference_full(wl)
+    assert np.array_equal(to_raw(ds.k_cache), k_ref)
+    assert np.array_equal(to_raw(ds.v_cache), v_ref)
+    assert_close(out, ref, wl.dtype, "tiny-mha")
+    assert int(ds.err.item()) == 0
+    # context length 1 (sequence 0) returns its new V exactly
+    for h in range(wl.num_heads):
+        assert np.array_equal(out[0, h], wl.v_new[0, h])
+
+
+# ------------------------------------------------------------------ sweep of small random cases
+
+SWEEP = [(dt, d, bs, g) for dt in ("f16", "bf16") for d in (64, 128) for bs in (8, 16, 32, 64) for g in (1, 2, 4, 8)]
+
+
+@pytest.mark.parametrize("dtype,head_dim,block_size,group", SWEEP,
+                         ids=[f"{a}-d{b}-bs{c}-g{d}" for a, b, c, d in SWEEP])
+def test_small_random_cases(dtype, head_dim, block_size, group):
+    kvh = 2
+    seed = 1000 + head_dim + block_size * 3 + group * 7 + (0 if dtype == "f16" else 500)
+    wl = inputs.random_case(seed, num_seqs=5, num_heads=kvh * group, num_kv_heads=kvh, head_dim=head_dim,
+                            block_size=block_size, dtype=dtype, ctx_lo=1, ctx_hi=300, table_filler=-2)
+    ds = DeviceState(wl, full_pool=True)
+    out = ds.step()
+    ref, k_ref, v_ref = reference_full(wl)
+    assert np.array_equal(to_raw(ds.k_cache), k_ref)
+    assert np.array_equal(to_raw(ds.v_cache), v_ref)
+    assert_close(out, ref, dtype, f"{dtype}-d{head_dim}-bs{block_size}-g{group}")
+    assert int(ds.err.item()) == 0
+
+
+@pytest.mark.parametrize("max_ctas", [1, 2, 3, 7, 0])
+def test_split_choice_does_not_change_the_result(max_ctas):
+    """Capping the grid changes where units are split (and how many partials
+    the merge combines); every choice must stay within tolerance."""
+    wl = inputs.random_case(77, num_seqs=6, num_heads=16, num_kv_heads=4, head_dim=128, block_size=16,
+                            dtype="bf16", ctx_lo=1, ctx_hi=3000)
+    ds = DeviceState(wl, full_pool=True)
+    out = ds.step(max_ctas=max_ctas)
+    ref, _, _ = reference_full(wl)
+    assert_close(out, ref, wl.dtype, f"max_ctas={max_ctas}")
+
+
+def test_many_short_sequences_and_empty_contexts():
+    """2048 sequences (the maximum) with contexts 0..40; empty ones give zeros."""
+    wl = inputs.random_case(5, num_seqs=2048, num_heads=4, num_kv_heads=4, head_dim=64, block_size=16,
+                            dtype="f16", ctx_lo=1, ctx_hi=40)
+    ctx = wl.context_lens.copy()
+    ctx[::7] = 0
+    wl.context_lens = ctx
+    wl.slot_mapping = np.where(ctx > 0, wl.slot_mapping, -1)
+    ds = DeviceState(wl, full_pool=True)
+    out = ds.step()
+    ref, k_ref, v_ref = reference_full(wl)
+    assert np.array_equal(to_raw(ds.k_cache), k_ref)
+    assert_close(out, ref, wl.dtype, "2048 seqs")
+    assert np.all(out[::7] == 0)
+
+
+# ------------------------------------------------------------------ full-size configs
+
+FULL = [1, 2, 4] + [("bs", b) for b in (8, 16, 32, 64)]
+
+
+def _full_workload(spec):
+    if isinstance(spec, tuple):
+        return inputs.config(3, block_size=spec[1])
+    return inputs.config(spec)
+
+
+@pytest.mark.parametrize("spec", FULL, ids=lambda s: f"llama13b-bs{s[1]}" if isinstance(s, tuple) else inputs.CONFIG_NAMES[s])
+def test_full_size_config(spec):
+    wl = _full_workload(spec)
+    ds = DeviceState(wl, full_pool=False)
+    k_before = ds.k_cache.clone()
+    v_before = ds.v_cache.clone()
+    out = ds.step()
+    assert int(ds.err.item()) == 0
+    # append: the new rows bit-exact, nothing else touched
+    slots = wl.slot_mapping
+    blk = torch.from_numpy(slots // wl.block_size).cuda()
+    off = torch.from_numpy(slots % wl.block_size).cuda()
+    assert torch.equal(ds.k_cache[blk, :, off, :].view(torch.int16), ds.k_new.view(torch.int16))
+    assert torch.equal(ds.v_cache[blk, :, off, :].view(torch.int16), ds.v_new.view(torch.int16))
+    k_after = ds.k_cache.clone()
+    v_after = ds.v_cache.clone()
+    k_after[blk, :, off, :] = 0
+    v_after[blk, :, off, :] = 0
+    k_before[blk, :, off, :] = 0
+    v_before[blk, :, off, :] = 0
+    assert torch.equal(k_after.view(torch.int16), k_before.view(torch.int16))
+    assert torch.equal(v_after.view(torch.int16), v_before.view(torch.int16))
+    del k_before, v_before, k_after, v_after
+    # decode: finite everywhere; sampled sequences/heads against the oracle
+    assert np.isfinite(oracle.widen(out, wl.dtype)).all()
+    ctx = wl.context_lens
+    seqs = sorted({0, wl.num_seqs - 1, int(np.argmax(ctx)), int(np.argmin(ctx)), wl.num_seqs // 2})
+    heads = sorted({0, wl.num_kv_heads - 1})
+    ref = reference_sampled(wl, seqs, heads)
+    for (s, h), r in ref.items():
+        assert_close(out[s, h], r, wl.dtype, f"{wl.name} seq {s} head {h}")
+
+
+# ------------------------------------------------------------------ invariants, bit for bit
+
+
+def test_permuting_physical_blocks_is_bit_identical():
+    wl = inputs.random_case(31, num_seqs=7, num_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                            dtype="f16", ctx_lo=1, ctx_hi=900)
+    out1 = DeviceState(wl, full_pool=True).step()
+    perm = np.random.default_rng(9).permutation(wl.num_blocks)
+    wl2 = inputs.random_case(31, num_seqs=7, num_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                             dtype="f16", ctx_lo=1, ctx_hi=900)
+    wl2.used = perm[wl.used]
+    nb = -(-wl.context_lens // 16)
+    t2 = wl.block_tables.copy()
+    for s in range(wl.num_seqs):
+        t2[s, : nb[s]] = perm[wl.block_tables[s, : nb[s]]]
+    wl2.block_tables = t2
+    wl2.slot_mapping = perm[wl.slot_mapping // 16] * 16 + wl.slot_mapping % 16
+    out2 = DeviceState(wl2, full_pool=True).step()
+    assert np.array_equal(out1, out2)
+
+
+def test_shared_prefix_equals_private_copies():
+    """Sequences whose tables point at the same prefix blocks give the same
+    bits as when each holds its own copy of those blocks."""
+    wl = inputs.build("prefix", seed=55, num_seqs=8, num_heads=64, num_kv_heads=8, head_dim=128, block_size=16,
+                      dtype="bf16", ctx_kind="uniform", ctx_lo=1100, ctx_hi=3000, shared_prefix_blocks=64,
+                      group_size=4, pool_factor=2.0)
+    out_shared = DeviceState(wl, full_pool=False).step()
+    # private copies: every sequence gets fresh blocks holding the prefix data
+    import copy
+
+    wl2 = copy.deepcopy(wl)
+    row_of = {int(p): i for i, p in enumerate(wl.used)}
+    free = [b for b in range(wl.num_blocks) if b not in row_of]
+    extra_k, extra_v, extra_ids = [], [], []
+    t2 = wl.block_tables.copy()
+    for s in range(wl.num_seqs):
+        if s % wl.group_size == 0:
+            continue
+        for i in range(wl.shared_prefix_blocks):
+            b = free.pop()
+            src = row_of[int(wl.block_tables[s, i])]
+            extra_ids.append(b)
+            extra_k.append(wl.k_blocks[src])
+            extra_v.append(wl.v_blocks[src])
+            t2[s, i] = b
+    wl2.block_tables = t2
+    wl2.used = np.concatenate([wl.used, np.array(extra_ids, dtype=np.int64)])
+    wl2.k_blocks = np.concatenate([wl.k_blocks, np.stack(extra_k)])
+    wl2.v_blocks = np.concatenate([wl.v_blocks, np.stack(extra_v)])
+    out_private = DeviceState(wl2, full_pool=False).step()
+    assert np.array_equal(out_shared, out_private)
+    ref = reference_sampled(wl, [0, 1, 5], [0, 7])
+    for (s, h), r in ref.items():
+        assert_close(out_shared[s, h], r, wl.dtype, f"prefix seq {s} head {h}")
+
+
+@pytest.mark.parametrize("dtype,group", [("f16", 1), ("bf16", 1), ("f16", 4), ("bf16", 8), ("f16", 2)])
+def test_context_one_returns_v_exactly(dtype, group):
+    wl = inputs.build("ctx1", seed=3, num_seqs=3, num_heads=2 * group, num_kv_heads=2, head_dim=128,
+                      block_size=16, dtype=dtype, context_lens=[1, 1, 1], pool_blocks=9)
+    out = DeviceState(wl, full_pool=True).step()
+    for s in range(3):
+        for h in range(2 * group):
+            assert np.array_equal(out[s, h], wl.v_new[s, h // group])
+
+
+@pytest.mark.parametrize("group", [1, 8])
+def test_dominant_key_selects_its_value(group):
+    """Key at one target position = 8 * q: its weight is ~1, so the output is
+    that position's V -- checks the table indexing of every target."""
+    wl = inputs.random_case(41, num_seqs=4, num_heads=2 * group, num_kv_heads=2, head_dim=64, block_size=8,
+                            dtype="f16", ctx_lo=40, ctx_hi=200)
+    k, v = wl.full_pool()
+    targets = []
+    for s in range(wl.num_seqs):
+        t = (s * 37) % (int(wl.context_lens[s]) - 1)
+        blk, off = int(wl.block_tables[s, t // 8]), t % 8
+        for h in range(2):
+            qv = wl.q[s, h * group].view(np.float16).astype(np.float32)
+            k[blk, h, off] = (qv * 8.0).astype(np.float16).view(np.uint16)
+        targets.append((s, blk, off))
+    ds = DeviceState(wl, full_pool=True)
+    ds.k_cache.copy_(to_dev(k, "f16"))
+    ds.v_cache.copy_(to_dev(v, "f16"))
+    out = ds.step()
+    for s, blk, off in targets:
+        for h in range(2):
+            got = oracle.widen(out[s, h * group], "f16")
+            want = v[blk, h, off].view(np.float16).astype(np.float64)
+            np.testing.assert_allclose(got, want, atol=2e-3, rtol=1e-2)
+
+
+# ------------------------------------------------------------------ error reporting without faults
+
+
+def test_out_of_range_ids_set_flags_and_stay_finite():
+    wl = inputs.random_case(8, num_seqs=4, num_heads=4, num_kv_heads=4, head_dim=128, block_size=16,
+                            dtype="f16", ctx_lo=20, ctx_hi=100)
+    ds = DeviceState(wl, full_pool=True)
+    bad_tables = ds.tables.clone()
+    bad_tables[2, 0] = wl.num_blocks + 5  # decode: skip that chunk, flag it
+    ds.tables = bad_tables
+    slots = ds.slots.clone()
+    slots[1] = wl.num_blocks * wl.block_size + 3  # append: skip that token, flag it
+    ds.slots = slots
+    out = ds.step()
+    flags = int(ds.err.item())
+    assert flags & libpaged.ERRF_BLOCK_RANGE
+    assert flags & libpaged.ERRF_SLOT_RANGE
+    # sequences 0 and 3 are untouched by the bad entries
+    ref, _, _ = reference_full(wl)
+    assert_close(out[[0, 3]], ref[[0, 3]], "f16", "good sequences")
+
+
+def test_context_above_bound_is_clamped_and_flagged():
+    wl = inputs.random_case(9, num_seqs=3, num_heads=2, num_kv_heads=2, head_dim=64, block_size=16,
+                            dtype="f16", ctx_lo=30, ctx_hi=60)
+    ds = DeviceState(wl, full_pool=True)
+    ds.append()
+    ds.err.zero_()
+    libpaged.decode(ds.out, ds.q, ds.k_cache, ds.v_cache, ds.tables, ds.ctx, float(wl.scale),
+                    max_context_len=int(wl.context_lens.min()) - 1, workspace=ds.ws, err_flags=ds.err)
+    torch.cuda.synchronize()
+    assert int(ds.err.item()) & libpaged.ERRF_CONTEXT
+    assert torch.isfinite(ds.out.float()).all()
+
+
+def test_status_codes_through_binding():
+    wl = inputs.random_case(10, num_seqs=2, num_heads=4, num_kv_heads=4, head_dim=64, block_size=16,
+                            dtype="f16", ctx_lo=5, ctx_hi=9)
+    ds = DeviceState(wl, full_pool=True)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(libpaged.LibpagedError) as e:
+        libpaged.decode(ds.out, ds.q, ds.k_cache, ds.v_cache, ds.tables, ds.ctx, 0.1, workspace=small)
+    assert e.value.status == libpaged.PA_ERR_WORKSPACE
