@@ -127,6 +127,10 @@ PA_API const char* pa_status_string(pa_status status);
 /* Library version, major*10000 + minor*100 + patch. */
 PA_API int pa_version(void);
 
+/* Detail of the last PA_ERR_CUDA / PA_ERR_UNSUPPORTED raised on this thread
+ * by a failing CUDA step (static thread-local storage; never NULL). */
+PA_API const char* pa_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -187,6 +187,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Host: record a failure detail for pa_last_error() and return `st`.
+pa_status fail(pa_status st, const char* what, cudaError_t e);
+
 __device__ __forceinline__ void set_err(int32_t* err, uint32_t bit) {
   if (err != nullptr) atomicOr(reinterpret_cast<unsigned int*>(err), bit);
 }

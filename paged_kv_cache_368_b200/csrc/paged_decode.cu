@@ -34,6 +34,7 @@
 //    the tensor cores (mma.sync m16n8k16, q-heads on M), fed by ldmatrix
 //    from the swizzled tiles.
 #include <algorithm>
+#include <cstdio>
 #include <atomic>
 #include <cmath>
 #include <mutex>
@@ -776,6 +777,19 @@ WsLayout ws_layout(int max_warps, int G, int D) {
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+}  // namespace
+
+namespace pa {
+thread_local char g_last_error[256] = "no error";
+
+pa_status fail(pa_status st, const char* what, cudaError_t e) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, e == cudaSuccess ? "" : cudaGetErrorString(e));
+  return st;
+}
+}  // namespace pa
+
+namespace {
+
 template <typename T, int D, int G>
 pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::DecodeParams& p, int ctas,
                         cudaStream_t stream, int dev) {
@@ -784,18 +798,27 @@ pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::
   static std::atomic<int> smem_set[kMaxDevices];
   const size_t smem = SH::smem_bytes(p.num_seqs);
   if (dev >= 0 && dev < kMaxDevices && smem_set[dev].load(std::memory_order_relaxed) < (int)smem) {
+    // Opt in to the largest dynamic size this kernel can use: the per-block
+    // limit minus the kernel's static shared memory.
     int optin = 0;
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if ((size_t)optin < smem) return PA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
-      return PA_ERR_CUDA;
-    smem_set[dev].store(optin, std::memory_order_relaxed);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "querying shared-memory limits", e);
+    const int dyn_max = optin - static_cast<int>(fa.sharedSizeBytes);
+    if (dyn_max < (int)smem) return pa::fail(PA_ERR_UNSUPPORTED, "num_seqs too large for shared memory", cudaSuccess);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max);
+    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaFuncSetAttribute(decode)", e);
+    smem_set[dev].store(dyn_max, std::memory_order_relaxed);
   }
   kern<<<ctas, pa::kWarps * 32, smem, stream>>>(km, vm, p);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_kernel", e);
   const int merge_blocks = (p.total_warps + 7) / 8;
   pa::paged_decode_merge_kernel<T, D, G><<<merge_blocks, 256, 0, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_merge_kernel", e);
+  return PA_OK;
 }
 
 template <typename T, int D>
@@ -854,9 +877,10 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (num_blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
 
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaGetDevice", ce);
   const int sms = device_sms(dev);
-  if (sms <= 0) return PA_ERR_CUDA;
+  if (sms <= 0) return pa::fail(PA_ERR_CUDA, "querying the SM count", cudaSuccess);
   const WsLayout L = ws_layout(sms * pa::kWarps, G, head_dim);
   if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return PA_ERR_WORKSPACE;
 
@@ -864,9 +888,10 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
 
   CUtensorMap km, vm;
+  if (!encode_fn()) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found", cudaSuccess);
   if (!make_cache_map(&km, k_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
       !make_cache_map(&vm, v_cache, num_blocks, num_kv_heads, block_size, head_dim))
-    return PA_ERR_CUDA;
+    return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled rejected the cache layout", cudaSuccess);
 
   pa::DecodeParams p;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -911,3 +936,5 @@ extern "C" const char* pa_status_string(pa_status status) {
 }
 
 extern "C" int pa_version(void) { return 100; }
+
+extern "C" const char* pa_last_error(void) { return pa::g_last_error; }

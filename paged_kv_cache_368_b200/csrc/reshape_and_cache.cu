@@ -75,5 +75,6 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, vo
       static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
       static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, vec_per_row, block_size,
       num_blocks * block_size, err_flags);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : pa::fail(PA_ERR_CUDA, "launching reshape_and_cache_kernel", e);
 }

@@ -24,7 +24,8 @@ ERRF_BLOCK_RANGE = 1 << 1
 ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
-SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_status_string", "pa_version")
+SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_status_string", "pa_version",
+           "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -35,7 +36,10 @@ _vp, _i32, _i64, _f32, _sz = _c.c_void_p, _c.c_int, _c.c_int64, _c.c_float, _c.c
 class LibpagedError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)}")
+        detail = ""
+        if status in (PA_ERR_CUDA, PA_ERR_UNSUPPORTED):
+            detail = " [" + load().pa_last_error().decode(errors="replace") + "]"
+        super().__init__(f"{where}: {status_string(status)}{detail}")
 
 
 def load(path: Optional[str] = None) -> ctypes.CDLL:
@@ -59,6 +63,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_status_string.restype = _c.c_char_p
     lib.pa_version.argtypes = []
     lib.pa_version.restype = _i32
+    lib.pa_last_error.argtypes = []
+    lib.pa_last_error.restype = _c.c_char_p
     if path is None:
         _lib = lib
     return lib
