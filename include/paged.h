@@ -121,6 +121,30 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype, void* workspace,
                     size_t workspace_bytes, int max_ctas, int32_t* err_flags, pa_stream_t stream);
 
+/*
+ * pa_decode_static -- pa_decode for callers that cannot allocate device
+ * memory (code where cudaMalloc is not allowed or not available, such as a
+ * host callback, a thread that must never block on an allocator, or a host
+ * application that hands a plugin only its input and output buffers).  The
+ * pages have no counterpart of this entry point; it exists for such callers.
+ *
+ * Same arguments and result as pa_decode, minus the workspace: the scratch
+ * is a 10 MiB array inside the library's device image, reserved on every
+ * GPU that uses this call until the process exits.  A shape that needs more
+ * scratch than that (pa_decode_workspace_size) returns PA_ERR_WORKSPACE; on
+ * a 148-SM B200 every supported shape fits.  All calls on one GPU share the
+ * array: calls that can run at the same time on that GPU race and give wrong
+ * results, so serialise them.  The array needs no clearing between calls.
+ * The first call on a device looks up the array's address
+ * (cudaGetSymbolAddress); make it before any stream capture on that device.
+ * Nothing is allocated or freed.
+ */
+PA_API pa_status pa_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                           int num_seqs, int max_context_len, float scale, int num_heads, int num_kv_heads,
+                           int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype, int max_ctas,
+                           int32_t* err_flags, pa_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 PA_API const char* pa_status_string(pa_status status);
 

@@ -24,8 +24,8 @@ ERRF_BLOCK_RANGE = 1 << 1
 ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
-SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_status_string", "pa_version",
-           "pa_last_error")
+SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_static",
+           "pa_status_string", "pa_version", "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -37,7 +37,7 @@ class LibpagedError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         detail = ""
-        if status in (PA_ERR_CUDA, PA_ERR_UNSUPPORTED):
+        if status in (PA_ERR_CUDA, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE):
             detail = " [" + load().pa_last_error().decode(errors="replace") + "]"
         super().__init__(f"{where}: {status_string(status)}{detail}")
 
@@ -59,6 +59,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64,
                               _i32, _vp, _sz, _i32, _vp, _vp]
     lib.pa_decode.restype = _i32
+    lib.pa_decode_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32, _i32, _i32,
+                                     _i64, _i32, _i32, _vp, _vp]
+    lib.pa_decode_static.restype = _i32
     lib.pa_status_string.argtypes = [_i32]
     lib.pa_status_string.restype = _c.c_char_p
     lib.pa_version.argtypes = []
@@ -169,4 +172,31 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
         _dev_ptr(err_flags, "err_flags"), _stream(stream))
     if st != PA_OK:
         raise LibpagedError(st, "pa_decode")
+    return out
+
+
+def decode_static(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                  max_context_len: Optional[int] = None, max_ctas: int = 0,
+                  err_flags: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """``decode`` without a workspace, for callers that cannot allocate device
+    memory: the library's own fixed 10 MiB scratch array is used instead.
+    Calls that may run concurrently on one GPU race on that array; make the
+    first call on a device before any stream capture."""
+    S, H, D = q.shape
+    nb, kvh, bs, _ = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q/out and the caches")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    mb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = mb * bs
+    st = load().pa_decode_static(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(block_tables, "block_tables"), mb, _dev_ptr(context_lens, "context_lens"), S,
+        int(max_context_len), float(scale), H, kvh, D, bs, nb, dtype_code(q.dtype), int(max_ctas),
+        _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_decode_static")
     return out
