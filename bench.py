@@ -135,6 +135,22 @@ def dist_init():
     return world, rank, local
 
 
+def reduce_max(value: float, dist, device) -> float:
+    """Max of a per-rank value over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput_gbs(bytes_per_step_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the bytes every rank processed over the slowest rank's time."""
+    return bytes_per_step_per_rank * world * steps / (max_ms * 1e-3) / 1e9
+
+
 def load_workload(args, poison=False):
     from paged_kv_cache_368_b200 import inputs
 
@@ -333,12 +349,8 @@ def run_ours(args):
         dist.barrier()
     if bad:
         raise SystemExit("libpaged call failed in the timed region")
-    elapsed_ms = e0.elapsed_time(e1)
+    elapsed_ms = reduce_max(e0.elapsed_time(e1), dist, dev)
     dec_ms = [a.elapsed_time(b) for a, b in dec]
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
 
     # ---- end to end through the public API: host buffers in, result out
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
@@ -351,17 +363,15 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_tables, h_ctx))
     d2h = h_out.numel() * h_out.element_size()
 
+    e_args = (h_q.data_ptr(), h_k.data_ptr(), h_v.data_ptr(), h_slots.data_ptr(), h_tables.data_ptr(),
+              h_ctx.data_ptr(), h_out.data_ptr(), q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
+              slots.data_ptr(), tables.data_ptr(), ctx.data_ptr(), out.data_ptr(), k_cache.data_ptr(),
+              v_cache.data_ptr(), wl.num_seqs, mb, max_ctx, float(wl.scale), wl.num_heads, kvh, D, bs, nb, code,
+              ws.data_ptr(), ws.numel(), err.data_ptr(), sp)
+
     def e2e_step():
-        q.copy_(h_q, non_blocking=True)
-        k_new.copy_(h_k, non_blocking=True)
-        v_new.copy_(h_v, non_blocking=True)
-        slots.copy_(h_slots, non_blocking=True)
-        tables.copy_(h_tables, non_blocking=True)
-        ctx.copy_(h_ctx, non_blocking=True)
-        libpaged.reshape_and_cache(k_new, v_new, k_cache, v_cache, slots, err_flags=err)
-        libpaged.decode(out, q, k_cache, v_cache, tables, ctx, float(wl.scale), max_context_len=max_ctx,
-                        workspace=ws, err_flags=err)
-        h_out.copy_(out, non_blocking=True)
+        if lib.pa_decode_step_host(*e_args) != 0:
+            raise SystemExit("pa_decode_step_host failed")
 
     Ke = min(K, 2000)
     for _ in range(max(3, W)):
@@ -375,15 +385,11 @@ def run_ours(args):
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = f0.elapsed_time(f1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(f0.elapsed_time(f1), dist, dev)
     clocks.stop()
 
     kvb = wl.kv_bytes()
-    value = kvb * world * K / (elapsed_ms * 1e-3) / 1e9
+    value = throughput_gbs(kvb, world, K, elapsed_ms)
     mean_dec = statistics.mean(dec_ms)
     achieved = kvb / (mean_dec * 1e-3) / 1e9
     peak, peak_src = measured_peak()
@@ -411,9 +417,9 @@ def run_ours(args):
                      "decode_us_mean": mean_dec * 1e3, "decode_us_median": statistics.median(dec_ms) * 1e3,
                      "decode_us_min": min(dec_ms) * 1e3, "kernel_src": src},
         "cpu_baseline": cpu,
-        "e2e": {"value": kvb * Ke / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": throughput_gbs(kvb, world, Ke, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke, "ms_per_step": e2e_ms / Ke,
-                "path": "pinned host -> device copies, libpaged.reshape_and_cache + libpaged.decode, device -> pinned host"},
+                "path": "pa_decode_step_host (C ABI): pinned host inputs -> device, append, decode, output -> pinned host"},
         "gpu_launches": 3 * K,
         "clocks": clocks.summary(t_wall0, t_wall1),
     }

@@ -122,6 +122,26 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     size_t workspace_bytes, int max_ctas, int32_t* err_flags, pa_stream_t stream);
 
 /*
+ * pa_decode_step_host -- one decode step whose per-step tensors live in host
+ * memory: copies q, key, value, slot_mapping, block_tables and context_lens
+ * from the h_* host buffers into the caller's d_* device buffers (same
+ * layouts as above; one new token per sequence, so num_tokens = num_seqs),
+ * runs pa_reshape_and_cache and pa_decode on the resident caches, and copies
+ * the output back into h_out.  Everything is enqueued on `stream` in that
+ * order; h_out is valid after the stream is synchronized.  Host buffers
+ * should be pinned (page-locked) for the copies to be asynchronous.  Errors
+ * are those of the two calls it makes, plus PA_ERR_CUDA for a failed copy.
+ */
+PA_API pa_status pa_decode_step_host(const void* h_q, const void* h_key, const void* h_value,
+                              const int64_t* h_slot_mapping, const int32_t* h_block_tables,
+                              const int32_t* h_context_lens, void* h_out, void* d_q, void* d_key, void* d_value,
+                              int64_t* d_slot_mapping, int32_t* d_block_tables, int32_t* d_context_lens,
+                              void* d_out, void* k_cache, void* v_cache, int num_seqs, int max_blocks_per_seq,
+                              int max_context_len, float scale, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int64_t num_blocks, pa_dtype dtype, void* workspace,
+                              size_t workspace_bytes, int32_t* err_flags, pa_stream_t stream);
+
+/*
  * pa_decode_static -- pa_decode for callers that cannot allocate device
  * memory (code where cudaMalloc is not allowed or not available, such as a
  * host callback, a thread that must never block on an allocator, or a host

@@ -67,6 +67,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Wait until the grids this one depends on have completed and their writes
+// are visible (a no-op when launched without programmatic serialization).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid in the stream to begin launching.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {

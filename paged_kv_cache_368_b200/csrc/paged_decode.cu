@@ -46,7 +46,31 @@ namespace pa {
 
 constexpr int kChunk = 16;       // tokens per pipeline stage
 constexpr int kMaxSeqs = 2048;   // prefix table lives in shared memory
-constexpr int kWarps = 8;        // warps per CTA
+#ifndef PA_CORE_WARPS
+#define PA_CORE_WARPS 8
+#endif
+#ifndef PA_CORE_DEPTH
+#define PA_CORE_DEPTH 2
+#endif
+#ifndef PA_MMA_WARPS
+#define PA_MMA_WARPS 6
+#endif
+#ifndef PA_MMA_DEPTH
+#define PA_MMA_DEPTH 2
+#endif
+#ifndef PA_D64_DEPTH
+#define PA_D64_DEPTH 4
+#endif
+
+// Warps per CTA and pipeline stages per warp for a shape (head_dim D, group G):
+// the per-warp ring of DEPTH stages must fit the 227 KB of shared memory.
+__host__ __device__ constexpr bool uses_mma(int G) { return G >= 4; }
+__host__ __device__ constexpr int warps_for(int D, int G) {
+  return D == 64 ? 8 : (uses_mma(G) ? PA_MMA_WARPS : PA_CORE_WARPS);
+}
+__host__ __device__ constexpr int depth_for(int D, int G) {
+  return D == 64 ? PA_D64_DEPTH : (uses_mma(G) ? PA_MMA_DEPTH : PA_CORE_DEPTH);
+}
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 struct DecodeParams {
@@ -73,8 +97,9 @@ struct DecodeParams {
 
 template <int D, int G>
 struct Shape {
-  static constexpr bool kMma = G >= 4;
-  static constexpr int kDepth = D == 64 ? 4 : (kMma ? 2 : 3);
+  static constexpr bool kMma = uses_mma(G);
+  static constexpr int kWarps = warps_for(D, G);
+  static constexpr int kDepth = depth_for(D, G);
   static constexpr int kTileBytes = kChunk * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQBytes = G * D * 2;
@@ -86,28 +111,24 @@ struct Shape {
 
 // --------------------------------------------------------------- chunk lookup
 
-struct ChunkInfo {
-  int seq;    // -1: no chunk
-  int head;   // kv-head
-  int c;      // chunk index inside the unit
-  int nc;     // chunks in the unit
-  int p0;     // physical block of the chunk's first rows
-  int p1;     // second physical block (block_size 8), or -1
-  int valid;  // tokens of the chunk inside the context; 0 = skip the chunk
-  int row0;   // first row of the chunk inside block p0
-};
-
 __device__ __forceinline__ int clamp_ctx(int ctx, int cap) { return ctx < 0 ? 0 : (ctx > cap ? cap : ctx); }
 
-// Chunk `g` of the global chunk order (g < total).  `prefix[s]` = chunks of
-// sequences < s, per kv-head.
-__device__ __forceinline__ ChunkInfo chunk_info(const DecodeParams& p, const int* prefix, int64_t g, int64_t end) {
-  ChunkInfo ci;
-  ci.seq = -1;
-  ci.head = ci.c = ci.nc = ci.p0 = ci.row0 = 0;
-  ci.p1 = -1;
-  ci.valid = 0;
-  if (g >= end) return ci;
+// Raw lookup of chunk `g` of the global chunk order: its unit and index from
+// the shared-memory prefix table, plus the three global words it needs
+// (context length and one or two block-table entries).  Windows of 32 chunks
+// are loaded one window ahead of use, so these loads never stall the warp.
+struct ChunkRaw {
+  int seq;  // -1: no chunk
+  int head, c, nc;
+  int ctx, p0, p1;
+};
+
+__device__ __forceinline__ ChunkRaw chunk_load(const DecodeParams& p, const int* prefix, int64_t g, int64_t end) {
+  ChunkRaw r;
+  r.seq = -1;
+  r.head = r.c = r.nc = r.ctx = r.p0 = 0;
+  r.p1 = -1;
+  if (g >= end) return r;
   const int KVH = p.num_kv_heads;
   int lo = 0, hi = p.num_seqs;  // largest s in [0, S) with KVH*prefix[s] <= g
   while (hi - lo > 1) {
@@ -119,43 +140,56 @@ __device__ __forceinline__ ChunkInfo chunk_info(const DecodeParams& p, const int
   const int rem = static_cast<int>(g - (int64_t)KVH * prefix[s]);
   const int h = rem / nc;
   const int c = rem - h * nc;
-  const int ctx = clamp_ctx(__ldg(p.context_lens + s), p.ctx_cap);
-  const int t0 = c * kChunk;
-  const int bs = p.block_size;
   const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-  int p0, p1 = -1, row0 = 0;
-  if (bs >= kChunk) {
-    p0 = __ldg(row + t0 / bs);
-    row0 = t0 % bs;
-  } else {  // two blocks of 8 tokens
-    p0 = __ldg(row + 2 * c);
-    if (t0 + 8 < ctx) p1 = __ldg(row + 2 * c + 1);
+  r.seq = s;
+  r.head = h;
+  r.c = c;
+  r.nc = nc;
+  r.ctx = __ldg(p.context_lens + s);
+  if (p.block_size >= kChunk) {
+    r.p0 = __ldg(row + c * kChunk / p.block_size);
+  } else {  // two blocks of 8 tokens; the second may lie past the context
+    r.p0 = __ldg(row + 2 * c);
+    if (2 * c + 1 < p.max_blocks_per_seq) r.p1 = __ldg(row + 2 * c + 1);
   }
-  bool ok = p0 >= 0 && p0 < p.num_blocks;
-  if (p1 != -1) ok = ok && p1 >= 0 && p1 < p.num_blocks;
-  if (!ok) set_err(p.err_flags, PA_ERRF_BLOCK_RANGE);
-  ci.seq = s;
-  ci.head = h;
-  ci.c = c;
-  ci.nc = nc;
-  ci.p0 = p0;
-  ci.p1 = ok ? p1 : -1;
-  ci.valid = ok ? min(kChunk, ctx - t0) : 0;
-  ci.row0 = row0;
-  return ci;
+  return r;
 }
 
-__device__ __forceinline__ ChunkInfo shfl_info(const ChunkInfo& a, int src) {
-  ChunkInfo r;
-  r.seq = __shfl_sync(kFull, a.seq, src);
-  r.head = __shfl_sync(kFull, a.head, src);
-  r.c = __shfl_sync(kFull, a.c, src);
-  r.nc = __shfl_sync(kFull, a.nc, src);
-  r.p0 = __shfl_sync(kFull, a.p0, src);
-  r.p1 = __shfl_sync(kFull, a.p1, src);
-  r.valid = __shfl_sync(kFull, a.valid, src);
-  r.row0 = __shfl_sync(kFull, a.row0, src);
-  return r;
+// Per-chunk words the warp shuffles around:
+//   sh    = seq | kv_head << 16
+//   flags = valid tokens (bits 0-4) | first row in the block (bits 5-10)
+//           | first chunk of its unit (bit 11) | last chunk of its unit (bit 12)
+//   p0/p1 = physical block(s); p1 = -1 when the chunk has one block.
+constexpr int kFlagStart = 1 << 11;
+constexpr int kFlagEnd = 1 << 12;
+
+struct ChunkInfo {
+  int sh, flags, p0, p1, c, nc;
+};
+
+__device__ __forceinline__ ChunkInfo chunk_finalize(const DecodeParams& p, const ChunkRaw& r) {
+  ChunkInfo ci;
+  ci.sh = ci.flags = ci.p0 = 0;
+  ci.p1 = -1;
+  ci.c = r.c;
+  ci.nc = r.nc;
+  if (r.seq < 0) return ci;
+  const int ctx = clamp_ctx(r.ctx, p.ctx_cap);
+  const int t0 = r.c * kChunk;
+  int valid = min(kChunk, ctx - t0);
+  int p1 = (p.block_size < kChunk && t0 + 8 < ctx) ? r.p1 : -1;
+  const bool ok = r.p0 >= 0 && r.p0 < p.num_blocks && (p1 == -1 || (p1 >= 0 && p1 < p.num_blocks));
+  if (!ok) {
+    set_err(p.err_flags, PA_ERRF_BLOCK_RANGE);
+    valid = 0;
+    p1 = -1;
+  }
+  const int row0 = p.block_size >= kChunk ? t0 % p.block_size : 0;
+  ci.sh = r.seq | (r.head << 16);
+  ci.flags = valid | (row0 << 5) | (r.c == 0 ? kFlagStart : 0) | (r.c == r.nc - 1 ? kFlagEnd : 0);
+  ci.p0 = r.p0;
+  ci.p1 = p1;
+  return ci;
 }
 
 // --------------------------------------------------------------- CUDA-core path
@@ -499,7 +533,7 @@ __device__ __forceinline__ void build_prefix(const DecodeParams& p, int* prefix)
 // --------------------------------------------------------------- main kernel
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kWarps * 32, 1)
+__global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                         const DecodeParams p) {
   using SH = Shape<D, G>;
@@ -516,9 +550,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   int* prefix = reinterpret_cast<int*>(bars + SH::kStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * kWarps + warp;
+  const int gw = blockIdx.x * SH::kWarps + warp;
   const int W = p.total_warps;
 
+  // Work that reads no global memory overlaps the previous kernel's tail
+  // (programmatic dependent launch); everything after griddep_wait sees all
+  // of its writes.
   if (threadIdx.x == 0) {
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
@@ -527,7 +564,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     for (int i = 0; i < DEPTH; ++i) mbar_init(&bars[warp * DEPTH + i], 1);
     fence_barrier_init();
   }
-  build_prefix<kWarps * 32>(p, prefix);
+  griddep_wait();
+  griddep_launch_dependents();
+  build_prefix<SH::kWarps * 32>(p, prefix);
   __syncthreads();
 
   const int S = p.num_seqs, H = p.num_heads;
@@ -535,6 +574,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_header[0] = static_cast<int>(NC);
   const int64_t c0 = (int64_t)gw * NC / W, c1 = (int64_t)(gw + 1) * NC / W;
   const int n = static_cast<int>(c1 - c0);
+
+  // Chunk windows: `cur` holds chunks [kb, kb+32), `nxt` [kb+32, kb+64), and
+  // the raw loads of [kb+64, kb+96) are in flight.
+  const ChunkRaw r0 = chunk_load(p, prefix, c0 + lane, c1);
+  const ChunkRaw r1 = chunk_load(p, prefix, c0 + 32 + lane, c1);
+  ChunkRaw rnext = chunk_load(p, prefix, c0 + 64 + lane, c1);
+  ChunkInfo cur = chunk_finalize(p, r0);
+  ChunkInfo nxt = chunk_finalize(p, r1);
+  int kb = 0;
 
   // Sequences with an empty context produce zeros.
   for (int s = gw; s < S; s += W) {
@@ -549,45 +597,47 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   const uint32_t box_bytes = rows_per_block * 128;
   const T* qbase = static_cast<const T*>(p.q);
 
-  ChunkInfo cur = chunk_info(p, prefix, c0 + lane, c1);
-  ChunkInfo nxt = chunk_info(p, prefix, c0 + 32 + lane, c1);
-  int kb = 0;  // chunk index held by lane 0 of `cur`
-
-  auto get = [&](int k) -> ChunkInfo {
+  // Issue the loads of chunk k into its stage (lane 0; all lanes shuffle).
+  auto issue = [&](int k) {
     const int d = k - kb;
-    return d < 32 ? shfl_info(cur, d) : shfl_info(nxt, d - 32);
-  };
-
-  auto issue = [&](int k, const ChunkInfo& ci) {
+    const bool in_cur = d < 32;
+    const int src = d & 31;
+    const int flags = __shfl_sync(kFull, in_cur ? cur.flags : nxt.flags, src);
+    const int sh = __shfl_sync(kFull, in_cur ? cur.sh : nxt.sh, src);
+    const int p0 = __shfl_sync(kFull, in_cur ? cur.p0 : nxt.p0, src);
+    const int p1 = __shfl_sync(kFull, in_cur ? cur.p1 : nxt.p1, src);
     if (lane != 0) return;
     const int stage = warp * DEPTH + (k % DEPTH);
     uint64_t* bar = &bars[stage];
-    const bool seg_start = (k == 0) || ci.c == 0;
-    const int nblk = ci.valid > 0 ? (ci.p1 >= 0 ? 2 : 1) : 0;
+    const bool seg_start = (k == 0) || (flags & kFlagStart);
+    const int valid = flags & 31;
+    const int row0 = (flags >> 5) & 63;
+    const int head = sh >> 16, seq = sh & 0xffff;
+    const int nblk = valid > 0 ? (p1 >= 0 ? 2 : 1) : 0;
     const uint32_t bytes = nblk * (D / 64) * box_bytes * 2 + (seg_start ? SH::kQBytes : 0);
     mbar_arrive_expect_tx(bar, bytes);
     const uint32_t kt = tiles + stage * SH::kStageBytes;
     const uint32_t vt = kt + SH::kTileBytes;
     for (int b = 0; b < nblk; ++b) {
-      const int phys = b == 0 ? ci.p0 : ci.p1;
+      const int phys = b == 0 ? p0 : p1;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const uint32_t off = c * 2048 + b * 1024;
-        tma_load_4d(kt + off, &kmap, bar, 64 * c, ci.row0, ci.head, phys, policy);
-        tma_load_4d(vt + off, &vmap, bar, 64 * c, ci.row0, ci.head, phys, policy);
+        tma_load_4d(kt + off, &kmap, bar, 64 * c, row0, head, phys, policy);
+        tma_load_4d(vt + off, &vmap, bar, 64 * c, row0, head, phys, policy);
       }
     }
     if (seg_start) {
-      const T* src = qbase + ((int64_t)ci.seq * H + (int64_t)ci.head * G) * D;
-      bulk_load(qslots + stage * SH::kQBytes, src, SH::kQBytes, bar);
+      const T* q_src = qbase + ((int64_t)seq * H + (int64_t)head * G) * D;
+      bulk_load(qslots + stage * SH::kQBytes, q_src, SH::kQBytes, bar);
     }
   };
 
-  for (int i = 0; i < DEPTH && i < n; ++i) issue(i, get(i));
+  for (int i = 0; i < DEPTH && i < n; ++i) issue(i);
 
   Warp st;
   st.reset();
-  int seg_first_c = 0;
+  bool seg_from_unit_start = false;
   bool first_seg = true;
   bool job_written = false;
   bool timed_out = false;
@@ -595,10 +645,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   for (; k < n; ++k) {
     if (k - kb >= 32) {
       cur = nxt;
+      nxt = chunk_finalize(p, rnext);
       kb += 32;
-      nxt = chunk_info(p, prefix, c0 + kb + 32 + lane, c1);
+      rnext = chunk_load(p, prefix, c0 + kb + 64 + lane, c1);
     }
-    const ChunkInfo ci = get(k);
+    const int d = k - kb;
+    const int flags = __shfl_sync(kFull, cur.flags, d);
+    const int sh = __shfl_sync(kFull, cur.sh, d);
     const int stage = warp * DEPTH + (k % DEPTH);
     const uint32_t parity = (k / DEPTH) & 1;
     // Every lane waits (acquiring the TMA writes); the give-up decision is
@@ -608,33 +661,35 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       timed_out = true;
       break;
     }
-    const bool seg_start = (k == 0) || ci.c == 0;
-    const bool seg_end = (k == n - 1) || ci.c == ci.nc - 1;
+    const bool seg_start = (k == 0) || (flags & kFlagStart);
+    const bool seg_end = (k == n - 1) || (flags & kFlagEnd);
     if (seg_start) {
       st.reset();
       st.load_q(qslots + stage * SH::kQBytes, p.scale_log2, lane);
-      seg_first_c = ci.c;
+      seg_from_unit_start = (flags & kFlagStart) != 0;
     }
+    const int valid = flags & 31;
     const uint32_t kt = tiles + stage * SH::kStageBytes;
     const uint32_t vt = kt + SH::kTileBytes;
-    if (ci.valid == kChunk) {
+    if (valid == kChunk) {
       if constexpr (SH::kMma) st.template chunk<false>(kt, vt, kChunk, lane, p.scale_log2);
       else st.template chunk<false>(kt, vt, kChunk, lane);
-    } else if (ci.valid > 0) {
+    } else if (valid > 0) {
       if constexpr (SH::kMma) {
-        zero_tail_rows<D>(vt, ci.valid, lane);
-        st.template chunk<true>(kt, vt, ci.valid, lane, p.scale_log2);
+        zero_tail_rows<D>(vt, valid, lane);
+        st.template chunk<true>(kt, vt, valid, lane, p.scale_log2);
       } else {
-        st.template chunk<true>(kt, vt, ci.valid, lane);
+        st.template chunk<true>(kt, vt, valid, lane);
       }
     }
     __syncwarp();
-    if (k + DEPTH < n) issue(k + DEPTH, get(k + DEPTH));
+    if (k + DEPTH < n) issue(k + DEPTH);
     if (seg_end) {
       st.finish();
-      const int kvh = ci.head;
-      if (seg_first_c == 0 && ci.c == ci.nc - 1) {
-        st.write_out(static_cast<T*>(p.out) + ((int64_t)ci.seq * H + (int64_t)kvh * G) * D, lane);
+      const int seq = sh & 0xffff, kvh = sh >> 16;
+      const bool unit_end = (flags & kFlagEnd) != 0;
+      if (seg_from_unit_start && unit_end) {
+        st.write_out(static_cast<T*>(p.out) + ((int64_t)seq * H + (int64_t)kvh * G) * D, lane);
       } else {
         const int slot = 2 * gw + (first_seg ? 0 : 1);
         st.write_partial(p.ws_o + (int64_t)slot * G * D, p.ws_ml + (int64_t)slot * G, lane);
@@ -642,10 +697,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       if (k == n - 1) {
         // The unit this warp's run ends in started here and continues in the
         // next warps: this warp owns its merge job.
+        const int c = __shfl_sync(kFull, cur.c, d);
+        const int nc = __shfl_sync(kFull, cur.nc, d);
         if (lane == 0) {
-          if (seg_first_c == 0 && ci.c < ci.nc - 1) {
-            const int64_t a = c0 + k - ci.c;
-            p.ws_jobs[gw] = make_int4(ci.seq, kvh, static_cast<int>(a), ci.nc);
+          if (seg_from_unit_start && !unit_end) {
+            const int64_t a = c0 + k - c;
+            p.ws_jobs[gw] = make_int4(seq, kvh, static_cast<int>(a), nc);
           } else {
             p.ws_jobs[gw] = make_int4(-1, 0, 0, 0);
           }
@@ -666,48 +723,124 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
 
 // --------------------------------------------------------------- merge kernel
 
-// Combines the partials of every unit that was split across warps:
+// Combines the partials of a unit split across warps w0..w1:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
-// (m in log2 units).  One warp per job.
+// (m in log2 units).  One CTA per merge job; its threads spread over the
+// contributing warps (for the max and the sum) and over (q-head, 4 output
+// columns) x groups of contributors (for the weighted sum), so the partial
+// loads are issued in parallel.
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
   using E = Elem<T>;
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  constexpr int ITEMS = G * D / 4;       // float4 outputs of one job
+  constexpr int NGRP = 256 / ITEMS;      // contributor groups
+  extern __shared__ int mslots[];        // [W] partial slot of each contributor, -1 if none
+  __shared__ float red[8][G];
+  __shared__ float sM[G], sL[G];
+  __shared__ float4 part[NGRP > 1 ? NGRP - 1 : 1][ITEMS];
+
+  griddep_wait();
+  griddep_launch_dependents();
   const int W = p.total_warps;
-  if (gw >= W) return;
-  const int4 job = p.ws_jobs[gw];
+  const int4 job = p.ws_jobs[blockIdx.x];
   if (job.x < 0) return;
   const int64_t NC = p.ws_header[0];
   const int64_t a = job.z, b = a + job.w;
-  auto start_of = [&](int64_t w) -> int64_t { return w * NC / W; };
-  const int64_t w_last = ((b - 1 + 1) * W + NC - 1) / NC - 1;  // warp holding chunk b-1
-  constexpr int PER = D / 32;
+  const int w0 = blockIdx.x;
+  const int w1 = static_cast<int>((b * W + NC - 1) / NC - 1);  // warp holding chunk b-1
+  const int nw = w1 - w0 + 1;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+
+  float mx[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
+  for (int j = t; j < nw; j += 256) {
+    const int64_t w = w0 + j;
+    const int64_t s0 = w * NC / W, s1 = (w + 1) * NC / W;
+    int slot = -1;
+    if (s0 < s1) {
+      slot = static_cast<int>(2 * w + (s0 >= a ? 0 : 1));
+#pragma unroll
+      for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], p.ws_ml[(int64_t)slot * G + g].x);
+    }
+    mslots[j] = slot;
+  }
+#pragma unroll
   for (int g = 0; g < G; ++g) {
-    float M = -INFINITY;
-    for (int64_t w = gw; w <= w_last; ++w) {
-      if (start_of(w) == start_of(w + 1)) continue;
-      const int64_t slot = 2 * w + (start_of(w) >= a ? 0 : 1);
-      M = fmaxf(M, p.ws_ml[slot * G + g].x);
+    float v = mx[g];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+    if (lane == 0) red[warp][g] = v;
+  }
+  __syncthreads();
+  if (t < G) {
+    float v = red[0][t];
+    for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w][t]);
+    sM[t] = v;
+  }
+  __syncthreads();
+  float sl[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) sl[g] = 0.f;
+  for (int j = t; j < nw; j += 256) {
+    const int slot = mslots[j];
+    if (slot < 0) continue;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float2 ml = p.ws_ml[(int64_t)slot * G + g];
+      if (ml.x != -INFINITY) sl[g] = fmaf(fast_exp2(ml.x - sM[g]), ml.y, sl[g]);
     }
-    float L = 0.f;
-    float acc[PER];
+  }
+  __syncthreads();  // red[] is reused
 #pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    for (int64_t w = gw; w <= w_last; ++w) {
-      if (start_of(w) == start_of(w + 1)) continue;
-      const int64_t slot = 2 * w + (start_of(w) >= a ? 0 : 1);
-      const float2 ml = p.ws_ml[slot * G + g];
-      const float e = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
-      L = fmaf(e, ml.y, L);
-      const float* po = p.ws_o + (slot * G + g) * D + lane * PER;
+  for (int g = 0; g < G; ++g) {
+    float v = sl[g];
 #pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = fmaf(e, po[i], acc[i]);
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    if (lane == 0) red[warp][g] = v;
+  }
+  __syncthreads();
+  if (t < G) {
+    float v = 0.f;
+    for (int w = 0; w < 8; ++w) v += red[w][t];
+    sL[t] = v;
+  }
+  __syncthreads();
+
+  const int item = t % ITEMS, grp = t / ITEMS;
+  const int g = item / (D / 4), d4 = item % (D / 4);
+  const float M = sM[g];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int j = grp; j < nw; j += NGRP) {
+    const int slot = mslots[j];
+    if (slot >= 0) {
+      const float m = p.ws_ml[(int64_t)slot * G + g].x;
+      const float4 o = reinterpret_cast<const float4*>(p.ws_o + ((int64_t)slot * G + g) * D)[d4];
+      const float e = m == -INFINITY ? 0.f : fast_exp2(m - M);
+      acc.x = fmaf(e, o.x, acc.x);
+      acc.y = fmaf(e, o.y, acc.y);
+      acc.z = fmaf(e, o.z, acc.z);
+      acc.w = fmaf(e, o.w, acc.w);
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    T* dst = static_cast<T*>(p.out) + ((int64_t)job.x * p.num_heads + (int64_t)job.y * G + g) * D + lane * PER;
+  }
+  if (NGRP > 1 && grp > 0) part[grp - 1][item] = acc;
+  __syncthreads();
+  if (grp == 0) {
 #pragma unroll
-    for (int i = 0; i < PER; i += 2) *reinterpret_cast<uint32_t*>(dst + i) = E::pack(acc[i] * inv, acc[i + 1] * inv);
+    for (int q = 1; q < NGRP; ++q) {
+      const float4 v = part[q - 1][item];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const float inv = sL[g] > 0.f ? 1.f / sL[g] : 0.f;
+    T* dst = static_cast<T*>(p.out) + ((int64_t)job.x * p.num_heads + (int64_t)job.y * G + g) * D + d4 * 4;
+    uint2 u;
+    u.x = E::pack(acc.x * inv, acc.y * inv);
+    u.y = E::pack(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(dst) = u;
   }
 }
 
@@ -811,12 +944,24 @@ pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::
     if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaFuncSetAttribute(decode)", e);
     smem_set[dev].store(dyn_max, std::memory_order_relaxed);
   }
-  kern<<<ctas, pa::kWarps * 32, smem, stream>>>(km, vm, p);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(SH::kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, p);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_kernel", e);
-  const int merge_blocks = (p.total_warps + 7) / 8;
-  pa::paged_decode_merge_kernel<T, D, G><<<merge_blocks, 256, 0, stream>>>(p);
-  e = cudaGetLastError();
+  // One CTA per warp of the decode grid (each may own a merge job).
+  cudaLaunchConfig_t mcfg = cfg;
+  mcfg.gridDim = dim3(p.total_warps);
+  mcfg.blockDim = dim3(256);
+  mcfg.dynamicSmemBytes = size_t(p.total_warps) * sizeof(int);
+  e = cudaLaunchKernelEx(&mcfg, pa::paged_decode_merge_kernel<T, D, G>, p);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_merge_kernel", e);
   return PA_OK;
 }
@@ -848,7 +993,7 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   const int sms = device_sms(dev);
   if (sms <= 0) return 0;
-  return ws_layout(sms * pa::kWarps, G, head_dim).total;
+  return ws_layout(sms * pa::warps_for(head_dim, G), G, head_dim).total;
 }
 
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -864,7 +1009,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (!valid_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-  if (num_seqs > pa::kMaxSeqs) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > pa::kMaxSeqs || num_kv_heads >= (1 << 15)) return PA_ERR_UNSUPPORTED;
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID;
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
@@ -881,10 +1026,11 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (ce != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaGetDevice", ce);
   const int sms = device_sms(dev);
   if (sms <= 0) return pa::fail(PA_ERR_CUDA, "querying the SM count", cudaSuccess);
-  const WsLayout L = ws_layout(sms * pa::kWarps, G, head_dim);
+  const int warps = pa::warps_for(head_dim, G);
+  const WsLayout L = ws_layout(sms * warps, G, head_dim);
   if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return PA_ERR_WORKSPACE;
 
-  int ctas = static_cast<int>(std::min<int64_t>(sms, std::max<int64_t>(1, (upper + pa::kWarps * 4 - 1) / (pa::kWarps * 4))));
+  int ctas = static_cast<int>(std::min<int64_t>(sms, std::max<int64_t>(1, (upper + warps * 4 - 1) / (warps * 4))));
   if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
 
   CUtensorMap km, vm;
@@ -912,7 +1058,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;
   p.block_size = block_size;
-  p.total_warps = ctas * pa::kWarps;
+  p.total_warps = ctas * warps;
   p.scale_log2 = scale * 1.4426950408889634f;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

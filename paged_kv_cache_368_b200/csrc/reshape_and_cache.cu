@@ -21,6 +21,10 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4* __r
                                                                  int64_t num_tokens, int num_kv_heads,
                                                                  int vec_per_row, int block_size,
                                                                  int64_t num_slots, int32_t* err_flags) {
+  // Launched with programmatic serialization: wait for the previous grid
+  // (which may still read the cache) before writing.
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t per_tensor = num_tokens * num_kv_heads * vec_per_row;
   const int64_t total = 2 * per_tensor;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
@@ -71,10 +75,18 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, vo
   const int threads = 256;
   const int64_t blocks64 = (total + threads - 1) / threads;
   const int blocks = static_cast<int>(blocks64 < 65535 ? blocks64 : 65535);
-  pa::reshape_and_cache_kernel<<<blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, vec_per_row, block_size,
-      num_blocks * block_size, err_flags);
-  const cudaError_t e = cudaGetLastError();
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, pa::reshape_and_cache_kernel, static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads,
+      vec_per_row, block_size, num_blocks * block_size, err_flags);
   return e == cudaSuccess ? PA_OK : pa::fail(PA_ERR_CUDA, "launching reshape_and_cache_kernel", e);
 }

@@ -25,7 +25,7 @@ ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
 SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_static",
-           "pa_status_string", "pa_version", "pa_last_error")
+           "pa_decode_step_host", "pa_status_string", "pa_version", "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -62,6 +62,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32, _i32, _i32,
                                      _i64, _i32, _i32, _vp, _vp]
     lib.pa_decode_static.restype = _i32
+    lib.pa_decode_step_host.argtypes = [_vp] * 16 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
+                                                     _vp, _sz, _vp, _vp]
+    lib.pa_decode_step_host.restype = _i32
     lib.pa_status_string.argtypes = [_i32]
     lib.pa_status_string.restype = _c.c_char_p
     lib.pa_version.argtypes = []
@@ -200,3 +203,41 @@ def decode_static(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_c
     if st != PA_OK:
         raise LibpagedError(st, "pa_decode_static")
     return out
+
+
+def _host_ptr(t: torch.Tensor, name: str) -> int:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def decode_step_host(h_q, h_key, h_value, h_slot_mapping, h_block_tables, h_context_lens, h_out,
+                     d_q, d_key, d_value, d_slot_mapping, d_block_tables, d_context_lens, d_out,
+                     k_cache, v_cache, scale: float, max_context_len: Optional[int] = None,
+                     workspace: Optional[torch.Tensor] = None, err_flags: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """One decode step from host tensors (pinned for asynchronous copies):
+    copy the inputs in, append the new K/V, decode, copy the output to
+    ``h_out``.  Returns ``h_out``; valid once the stream is synchronized."""
+    S, H, D = h_q.shape
+    nb, kvh, bs, _ = k_cache.shape
+    mb = h_block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = mb * bs
+    if workspace is None:
+        workspace = alloc_workspace(S, H, kvh, D, max_context_len, device=k_cache.device)
+    st = load().pa_decode_step_host(
+        _host_ptr(h_q, "h_q"), _host_ptr(h_key, "h_key"), _host_ptr(h_value, "h_value"),
+        _host_ptr(h_slot_mapping, "h_slot_mapping"), _host_ptr(h_block_tables, "h_block_tables"),
+        _host_ptr(h_context_lens, "h_context_lens"), _host_ptr(h_out, "h_out"),
+        _dev_ptr(d_q, "d_q"), _dev_ptr(d_key, "d_key"), _dev_ptr(d_value, "d_value"),
+        _dev_ptr(d_slot_mapping, "d_slot_mapping"), _dev_ptr(d_block_tables, "d_block_tables"),
+        _dev_ptr(d_context_lens, "d_context_lens"), _dev_ptr(d_out, "d_out"),
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), S, mb, int(max_context_len), float(scale),
+        H, kvh, D, bs, nb, dtype_code(h_q.dtype), _dev_ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_decode_step_host")
+    return h_out

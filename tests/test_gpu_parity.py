@@ -272,3 +272,32 @@ def test_status_codes_through_binding():
     with pytest.raises(libpaged.LibpagedError) as e:
         libpaged.decode(ds.out, ds.q, ds.k_cache, ds.v_cache, ds.tables, ds.ctx, 0.1, workspace=small)
     assert e.value.status == libpaged.PA_ERR_WORKSPACE
+
+
+def test_decode_step_from_host_buffers():
+    """pa_decode_step_host (copies in, append, decode, copy out) gives the same
+    bits as the device-resident calls, and matches the oracle."""
+    wl = inputs.random_case(71, num_seqs=6, num_heads=16, num_kv_heads=4, head_dim=128, block_size=16,
+                            dtype="bf16", ctx_lo=1, ctx_hi=1500)
+    ds = DeviceState(wl, full_pool=True)
+    dev_out = ds.step()
+    ds2 = DeviceState(wl, full_pool=True)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+    h_q = pin(wl.q.view(np.int16)).view(torch.bfloat16)
+    h_k = pin(wl.k_new.view(np.int16)).view(torch.bfloat16)
+    h_v = pin(wl.v_new.view(np.int16)).view(torch.bfloat16)
+    h_out = torch.empty_like(h_q).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(ds2.q), torch.empty_like(ds2.k_new), torch.empty_like(ds2.v_new)
+    d_slots, d_tables, d_ctx = torch.empty_like(ds2.slots), torch.empty_like(ds2.tables), torch.empty_like(ds2.ctx)
+    libpaged.decode_step_host(h_q, h_k, h_v, pin(wl.slot_mapping.astype(np.int64)),
+                              pin(wl.block_tables.astype(np.int32)), pin(wl.context_lens.astype(np.int32)), h_out,
+                              d_q, d_k, d_v, d_slots, d_tables, d_ctx, torch.empty_like(ds2.q),
+                              ds2.k_cache, ds2.v_cache, float(wl.scale), max_context_len=wl.max_context_len,
+                              workspace=ds2.ws, err_flags=ds2.err)
+    torch.cuda.synchronize()
+    host_out = h_out.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(host_out, dev_out)
+    assert np.array_equal(to_raw(ds2.k_cache), to_raw(ds.k_cache))
+    ref, _, _ = reference_full(wl)
+    assert_close(host_out, ref, wl.dtype, "host step")
+    assert int(ds2.err.item()) == 0
