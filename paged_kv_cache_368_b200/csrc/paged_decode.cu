@@ -725,19 +725,18 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
 
 // Combines the partials of a unit split across warps w0..w1:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
-// (m in log2 units).  One CTA per merge job; its threads spread over the
-// contributing warps (for the max and the sum) and over (q-head, 4 output
-// columns) x groups of contributors (for the weighted sum), so the partial
-// loads are issued in parallel.
+// (m in log2 units).  One CTA per merge job.  Thread (group, item) folds the
+// contributors j = group, group + NGRP, ... of one (q-head, 4 columns) item
+// into a running (m, l, acc) -- the same online rescaling as the decode
+// kernel -- so all partial loads of a thread are independent and issued
+// together; the NGRP groups are then combined once through shared memory.
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
   using E = Elem<T>;
-  constexpr int ITEMS = G * D / 4;       // float4 outputs of one job
-  constexpr int NGRP = 256 / ITEMS;      // contributor groups
-  extern __shared__ int mslots[];        // [W] partial slot of each contributor, -1 if none
-  __shared__ float red[8][G];
-  __shared__ float sM[G], sL[G];
-  __shared__ float4 part[NGRP > 1 ? NGRP - 1 : 1][ITEMS];
+  constexpr int ITEMS = G * D / 4;   // float4 outputs of one job
+  constexpr int NGRP = 256 / ITEMS;  // contributor groups
+  __shared__ float4 s_acc[256];
+  __shared__ float2 s_ml[256];
 
   griddep_wait();
   griddep_launch_dependents();
@@ -749,99 +748,57 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int w0 = blockIdx.x;
   const int w1 = static_cast<int>((b * W + NC - 1) / NC - 1);  // warp holding chunk b-1
   const int nw = w1 - w0 + 1;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-
-  float mx[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
-  for (int j = t; j < nw; j += 256) {
-    const int64_t w = w0 + j;
-    const int64_t s0 = w * NC / W, s1 = (w + 1) * NC / W;
-    int slot = -1;
-    if (s0 < s1) {
-      slot = static_cast<int>(2 * w + (s0 >= a ? 0 : 1));
-#pragma unroll
-      for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], p.ws_ml[(int64_t)slot * G + g].x);
-    }
-    mslots[j] = slot;
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float v = mx[g];
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
-    if (lane == 0) red[warp][g] = v;
-  }
-  __syncthreads();
-  if (t < G) {
-    float v = red[0][t];
-    for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w][t]);
-    sM[t] = v;
-  }
-  __syncthreads();
-  float sl[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) sl[g] = 0.f;
-  for (int j = t; j < nw; j += 256) {
-    const int slot = mslots[j];
-    if (slot < 0) continue;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float2 ml = p.ws_ml[(int64_t)slot * G + g];
-      if (ml.x != -INFINITY) sl[g] = fmaf(fast_exp2(ml.x - sM[g]), ml.y, sl[g]);
-    }
-  }
-  __syncthreads();  // red[] is reused
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float v = sl[g];
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-    if (lane == 0) red[warp][g] = v;
-  }
-  __syncthreads();
-  if (t < G) {
-    float v = 0.f;
-    for (int w = 0; w < 8; ++w) v += red[w][t];
-    sL[t] = v;
-  }
-  __syncthreads();
-
+  const int t = threadIdx.x;
   const int item = t % ITEMS, grp = t / ITEMS;
   const int g = item / (D / 4), d4 = item % (D / 4);
-  const float M = sM[g];
+
+  float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int j = grp; j < nw; j += NGRP) {
-    const int slot = mslots[j];
-    if (slot >= 0) {
-      const float m = p.ws_ml[(int64_t)slot * G + g].x;
-      const float4 o = reinterpret_cast<const float4*>(p.ws_o + ((int64_t)slot * G + g) * D)[d4];
-      const float e = m == -INFINITY ? 0.f : fast_exp2(m - M);
-      acc.x = fmaf(e, o.x, acc.x);
-      acc.y = fmaf(e, o.y, acc.y);
-      acc.z = fmaf(e, o.z, acc.z);
-      acc.w = fmaf(e, o.w, acc.w);
+    const int64_t w = w0 + j;
+    const int64_t s0 = w * NC / W, s1 = (w + 1) * NC / W;
+    if (s0 < s1) {  // warps with an empty run wrote nothing
+      const int64_t slot = 2 * w + (s0 >= a ? 0 : 1);
+      const float2 ml = p.ws_ml[slot * G + g];
+      const float4 o = reinterpret_cast<const float4*>(p.ws_o + (slot * G + g) * D)[d4];
+      if (ml.x != -INFINITY) {
+        const float mn = fmaxf(m, ml.x);
+        const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
+        l = l * sa + ml.y * sb;
+        acc.x = acc.x * sa + o.x * sb;
+        acc.y = acc.y * sa + o.y * sb;
+        acc.z = acc.z * sa + o.z * sb;
+        acc.w = acc.w * sa + o.w * sb;
+        m = mn;
+      }
     }
   }
-  if (NGRP > 1 && grp > 0) part[grp - 1][item] = acc;
-  __syncthreads();
-  if (grp == 0) {
-#pragma unroll
+  if (NGRP > 1) {
+    s_acc[t] = acc;
+    s_ml[t] = make_float2(m, l);
+    __syncthreads();
+    if (grp != 0) return;
     for (int q = 1; q < NGRP; ++q) {
-      const float4 v = part[q - 1][item];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+      const float2 ml = s_ml[q * ITEMS + item];
+      if (ml.x == -INFINITY) continue;
+      const float4 o = s_acc[q * ITEMS + item];
+      const float mn = fmaxf(m, ml.x);
+      const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
+      l = l * sa + ml.y * sb;
+      acc.x = acc.x * sa + o.x * sb;
+      acc.y = acc.y * sa + o.y * sb;
+      acc.z = acc.z * sa + o.z * sb;
+      acc.w = acc.w * sa + o.w * sb;
+      m = mn;
     }
-    const float inv = sL[g] > 0.f ? 1.f / sL[g] : 0.f;
-    T* dst = static_cast<T*>(p.out) + ((int64_t)job.x * p.num_heads + (int64_t)job.y * G + g) * D + d4 * 4;
-    uint2 u;
-    u.x = E::pack(acc.x * inv, acc.y * inv);
-    u.y = E::pack(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(dst) = u;
   }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  T* dst = static_cast<T*>(p.out) + ((int64_t)job.x * p.num_heads + (int64_t)job.y * G + g) * D + d4 * 4;
+  uint2 u;
+  u.x = E::pack(acc.x * inv, acc.y * inv);
+  u.y = E::pack(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(dst) = u;
 }
 
 }  // namespace pa
@@ -960,7 +917,7 @@ pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::
   cudaLaunchConfig_t mcfg = cfg;
   mcfg.gridDim = dim3(p.total_warps);
   mcfg.blockDim = dim3(256);
-  mcfg.dynamicSmemBytes = size_t(p.total_warps) * sizeof(int);
+  mcfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&mcfg, pa::paged_decode_merge_kernel<T, D, G>, p);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_merge_kernel", e);
   return PA_OK;
