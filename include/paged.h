@@ -122,24 +122,32 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     size_t workspace_bytes, int max_ctas, int32_t* err_flags, pa_stream_t stream);
 
 /*
- * pa_decode_step_host -- one decode step whose per-step tensors live in host
- * memory: copies q, key, value, slot_mapping, block_tables and context_lens
- * from the h_* host buffers into the caller's d_* device buffers (same
- * layouts as above; one new token per sequence, so num_tokens = num_seqs),
- * runs pa_reshape_and_cache and pa_decode on the resident caches, and copies
- * the output back into h_out.  Everything is enqueued on `stream` in that
- * order; h_out is valid after the stream is synchronized.  Host buffers
+ * pa_step_inputs_layout -- where each per-step input sits in the packed
+ * staging buffer of pa_decode_step_host.  Writes the byte offsets of q, key,
+ * value, slot_mapping, block_tables and context_lens (in that order, each
+ * 256-byte aligned, layouts as above, one new token per sequence) to
+ * offsets[0..5] and returns the buffer's total size (0 for bad arguments).
+ */
+PA_API size_t pa_step_inputs_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                    int max_blocks_per_seq, size_t offsets[6]);
+
+/*
+ * pa_decode_step_host -- one decode step whose per-step inputs live in host
+ * memory.  h_inputs holds q, key, value, slot_mapping, block_tables and
+ * context_lens packed as pa_step_inputs_layout describes; it is copied in one
+ * piece into the caller's device staging buffer d_inputs (same size,
+ * 256-byte aligned), then pa_reshape_and_cache and pa_decode run on the
+ * resident caches (output in d_out, [num_seqs][num_heads][head_dim]) and the
+ * output is copied back into h_out.  Everything is enqueued on `stream` in
+ * that order; h_out is valid after the stream is synchronized.  Host buffers
  * should be pinned (page-locked) for the copies to be asynchronous.  Errors
  * are those of the two calls it makes, plus PA_ERR_CUDA for a failed copy.
  */
-PA_API pa_status pa_decode_step_host(const void* h_q, const void* h_key, const void* h_value,
-                              const int64_t* h_slot_mapping, const int32_t* h_block_tables,
-                              const int32_t* h_context_lens, void* h_out, void* d_q, void* d_key, void* d_value,
-                              int64_t* d_slot_mapping, int32_t* d_block_tables, int32_t* d_context_lens,
-                              void* d_out, void* k_cache, void* v_cache, int num_seqs, int max_blocks_per_seq,
-                              int max_context_len, float scale, int num_heads, int num_kv_heads, int head_dim,
-                              int block_size, int64_t num_blocks, pa_dtype dtype, void* workspace,
-                              size_t workspace_bytes, int32_t* err_flags, pa_stream_t stream);
+PA_API pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, void* h_out, void* d_out, void* k_cache,
+                              void* v_cache, int num_seqs, int max_blocks_per_seq, int max_context_len,
+                              float scale, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                              int64_t num_blocks, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                              int32_t* err_flags, pa_stream_t stream);
 
 /*
  * pa_decode_static -- pa_decode for callers that cannot allocate device

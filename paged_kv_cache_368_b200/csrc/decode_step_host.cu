@@ -5,53 +5,67 @@
 // ("【infra之路】10-PagedAttention 与 KV Cache 管理": append, then attend).
 //
 // The KV caches and the workspace stay resident on the device; only the
-// per-step tensors cross PCIe.  One cudaMemcpyAsync per tensor (host buffers
-// should be pinned for the copies to be asynchronous).
+// per-step tensors cross PCIe.  They travel packed in one staging buffer
+// (layout from pa_step_inputs_layout), so a step costs one host-to-device
+// and one device-to-host copy.
 #include "pa_device.cuh"
 
-extern "C" pa_status pa_decode_step_host(const void* h_q, const void* h_key, const void* h_value,
-                                         const int64_t* h_slot_mapping, const int32_t* h_block_tables,
-                                         const int32_t* h_context_lens, void* h_out, void* d_q, void* d_key,
-                                         void* d_value, int64_t* d_slot_mapping, int32_t* d_block_tables,
-                                         int32_t* d_context_lens, void* d_out, void* k_cache, void* v_cache,
-                                         int num_seqs, int max_blocks_per_seq, int max_context_len, float scale,
-                                         int num_heads, int num_kv_heads, int head_dim, int block_size,
-                                         int64_t num_blocks, pa_dtype dtype, void* workspace,
-                                         size_t workspace_bytes, int32_t* err_flags, pa_stream_t stream) {
-  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0)
-    return PA_ERR_INVALID;
-  if (num_seqs == 0) return PA_OK;
-  if (!h_q || !h_key || !h_value || !h_slot_mapping || !h_block_tables || !h_context_lens || !h_out || !d_q ||
-      !d_key || !d_value || !d_slot_mapping || !d_block_tables || !d_context_lens || !d_out)
-    return PA_ERR_INVALID;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+namespace {
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+}  // namespace
+
+extern "C" size_t pa_step_inputs_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                        int max_blocks_per_seq, size_t offsets[6]) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || !offsets)
+    return 0;
   const size_t S = static_cast<size_t>(num_seqs);
-  const size_t q_bytes = S * num_heads * head_dim * 2;
-  const size_t kv_bytes = S * num_kv_heads * head_dim * 2;
-  struct Copy {
-    void* dst;
-    const void* src;
-    size_t bytes;
-  } in[] = {
-      {d_key, h_key, kv_bytes},
-      {d_value, h_value, kv_bytes},
-      {d_slot_mapping, h_slot_mapping, S * sizeof(int64_t)},
-      {d_q, h_q, q_bytes},
-      {d_block_tables, h_block_tables, S * max_blocks_per_seq * sizeof(int32_t)},
-      {d_context_lens, h_context_lens, S * sizeof(int32_t)},
+  const size_t sizes[6] = {
+      S * num_heads * head_dim * 2,           // q
+      S * num_kv_heads * head_dim * 2,        // key
+      S * num_kv_heads * head_dim * 2,        // value
+      S * sizeof(int64_t),                    // slot_mapping
+      S * max_blocks_per_seq * sizeof(int32_t),  // block_tables
+      S * sizeof(int32_t),                    // context_lens
   };
-  for (const Copy& c : in) {
-    const cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host: host-to-device copy", e);
+  size_t off = 0;
+  for (int i = 0; i < 6; ++i) {
+    offsets[i] = off;
+    off = align256(off + sizes[i]);
   }
-  pa_status st = pa_reshape_and_cache(d_key, d_value, k_cache, v_cache, d_slot_mapping, num_seqs, num_kv_heads,
-                                      head_dim, block_size, num_blocks, dtype, err_flags, stream);
+  return off;
+}
+
+extern "C" pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, void* h_out, void* d_out,
+                                         void* k_cache, void* v_cache, int num_seqs, int max_blocks_per_seq,
+                                         int max_context_len, float scale, int num_heads, int num_kv_heads,
+                                         int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                                         void* workspace, size_t workspace_bytes, int32_t* err_flags,
+                                         pa_stream_t stream) {
+  size_t off[6];
+  const size_t total = pa_step_inputs_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq, off);
+  if (total == 0) return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!h_inputs || !d_inputs || !h_out || !d_out) return PA_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(d_inputs) & 255u) return PA_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(d_inputs, h_inputs, total, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host: host-to-device copy", e);
+  uint8_t* d = static_cast<uint8_t*>(d_inputs);
+  const void* d_q = d + off[0];
+  const void* d_key = d + off[1];
+  const void* d_value = d + off[2];
+  const int64_t* d_slots = reinterpret_cast<const int64_t*>(d + off[3]);
+  const int32_t* d_tables = reinterpret_cast<const int32_t*>(d + off[4]);
+  const int32_t* d_ctx = reinterpret_cast<const int32_t*>(d + off[5]);
+  pa_status st = pa_reshape_and_cache(d_key, d_value, k_cache, v_cache, d_slots, num_seqs, num_kv_heads, head_dim,
+                                      block_size, num_blocks, dtype, err_flags, stream);
   if (st != PA_OK) return st;
-  st = pa_decode(d_out, d_q, k_cache, v_cache, d_block_tables, max_blocks_per_seq, d_context_lens, num_seqs,
-                 max_context_len, scale, num_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype, workspace,
-                 workspace_bytes, 0, err_flags, stream);
+  st = pa_decode(d_out, d_q, k_cache, v_cache, d_tables, max_blocks_per_seq, d_ctx, num_seqs, max_context_len, scale,
+                 num_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype, workspace, workspace_bytes, 0,
+                 err_flags, stream);
   if (st != PA_OK) return st;
-  const cudaError_t e = cudaMemcpyAsync(h_out, d_out, q_bytes, cudaMemcpyDeviceToHost, s);
+  const size_t out_bytes = static_cast<size_t>(num_seqs) * num_heads * head_dim * 2;
+  e = cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host: device-to-host copy", e);
   return PA_OK;
 }

@@ -723,20 +723,38 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
 
 // --------------------------------------------------------------- merge kernel
 
+// Threads of one merge CTA: enough that every (q-head, 4 columns) item has
+// several threads sharing out the contributors.
+__host__ __device__ constexpr int merge_threads(int D, int G) { return G * D / 4 >= 128 ? 1024 : 256; }
+
+// One online-softmax fold of a partial (ml, o) into the running (m, l, acc).
+__device__ __forceinline__ void fold_partial(float& m, float& l, float4& acc, float2 ml, float4 o) {
+  const float mn = fmaxf(m, ml.x);
+  const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
+  l = l * sa + ml.y * sb;
+  acc.x = acc.x * sa + o.x * sb;
+  acc.y = acc.y * sa + o.y * sb;
+  acc.z = acc.z * sa + o.z * sb;
+  acc.w = acc.w * sa + o.w * sb;
+  m = mn;
+}
+
 // Combines the partials of a unit split across warps w0..w1:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
-// (m in log2 units).  One CTA per merge job.  Thread (group, item) folds the
+// (m in log2 units).  One CTA per merge job.  The contributors' partial
+// slots are resolved once into shared memory; thread (group, item) then folds
 // contributors j = group, group + NGRP, ... of one (q-head, 4 columns) item
-// into a running (m, l, acc) -- the same online rescaling as the decode
-// kernel -- so all partial loads of a thread are independent and issued
-// together; the NGRP groups are then combined once through shared memory.
+// into a running (m, l, acc), loading four contributors at a time, and the
+// NGRP groups are combined once through shared memory.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(merge_threads(D, G)) paged_decode_merge_kernel(const DecodeParams p) {
   using E = Elem<T>;
-  constexpr int ITEMS = G * D / 4;   // float4 outputs of one job
-  constexpr int NGRP = 256 / ITEMS;  // contributor groups
-  __shared__ float4 s_acc[256];
-  __shared__ float2 s_ml[256];
+  constexpr int NT = merge_threads(D, G);
+  constexpr int ITEMS = G * D / 4;  // float4 outputs of one job
+  constexpr int NGRP = NT / ITEMS;  // contributor groups
+  extern __shared__ int mslots[];   // [W]: partial slot of each contributor, -1 if it has none
+  __shared__ float4 s_acc[NT];
+  __shared__ float2 s_ml[NT];
 
   griddep_wait();
   griddep_launch_dependents();
@@ -749,30 +767,40 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int w1 = static_cast<int>((b * W + NC - 1) / NC - 1);  // warp holding chunk b-1
   const int nw = w1 - w0 + 1;
   const int t = threadIdx.x;
+  for (int j = t; j < nw; j += NT) {
+    const int64_t w = w0 + j;
+    const int64_t s0 = w * NC / W, s1 = (w + 1) * NC / W;  // warps with an empty run wrote nothing
+    mslots[j] = s0 < s1 ? static_cast<int>(2 * w + (s0 >= a ? 0 : 1)) : -1;
+  }
+  __syncthreads();
+
   const int item = t % ITEMS, grp = t / ITEMS;
   const int g = item / (D / 4), d4 = item % (D / 4);
-
+  auto ml_at = [&](int slot) { return p.ws_ml[(int64_t)slot * G + g]; };
+  auto o_at = [&](int slot) { return reinterpret_cast<const float4*>(p.ws_o + ((int64_t)slot * G + g) * D)[d4]; };
   float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int j = grp; j < nw; j += NGRP) {
-    const int64_t w = w0 + j;
-    const int64_t s0 = w * NC / W, s1 = (w + 1) * NC / W;
-    if (s0 < s1) {  // warps with an empty run wrote nothing
-      const int64_t slot = 2 * w + (s0 >= a ? 0 : 1);
-      const float2 ml = p.ws_ml[slot * G + g];
-      const float4 o = reinterpret_cast<const float4*>(p.ws_o + (slot * G + g) * D)[d4];
-      if (ml.x != -INFINITY) {
-        const float mn = fmaxf(m, ml.x);
-        const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
-        l = l * sa + ml.y * sb;
-        acc.x = acc.x * sa + o.x * sb;
-        acc.y = acc.y * sa + o.y * sb;
-        acc.z = acc.z * sa + o.z * sb;
-        acc.w = acc.w * sa + o.w * sb;
-        m = mn;
-      }
+  int j = grp;
+  for (; j + 3 * NGRP < nw; j += 4 * NGRP) {
+    int sl[4];
+    float2 ml[4];
+    float4 o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      sl[u] = mslots[j + u * NGRP];
+      const int safe = sl[u] < 0 ? 0 : sl[u];  // a valid address; its values are not used
+      ml[u] = ml_at(safe);
+      o[u] = o_at(safe);
     }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (sl[u] >= 0 && ml[u].x != -INFINITY) fold_partial(m, l, acc, ml[u], o[u]);
+  }
+  for (; j < nw; j += NGRP) {
+    const int slot = mslots[j];
+    if (slot < 0) continue;
+    const float2 ml = ml_at(slot);
+    if (ml.x != -INFINITY) fold_partial(m, l, acc, ml, o_at(slot));
   }
   if (NGRP > 1) {
     s_acc[t] = acc;
@@ -781,16 +809,7 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
     if (grp != 0) return;
     for (int q = 1; q < NGRP; ++q) {
       const float2 ml = s_ml[q * ITEMS + item];
-      if (ml.x == -INFINITY) continue;
-      const float4 o = s_acc[q * ITEMS + item];
-      const float mn = fmaxf(m, ml.x);
-      const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
-      l = l * sa + ml.y * sb;
-      acc.x = acc.x * sa + o.x * sb;
-      acc.y = acc.y * sa + o.y * sb;
-      acc.z = acc.z * sa + o.z * sb;
-      acc.w = acc.w * sa + o.w * sb;
-      m = mn;
+      if (ml.x != -INFINITY) fold_partial(m, l, acc, ml, s_acc[q * ITEMS + item]);
     }
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -916,8 +935,8 @@ pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::
   // One CTA per warp of the decode grid (each may own a merge job).
   cudaLaunchConfig_t mcfg = cfg;
   mcfg.gridDim = dim3(p.total_warps);
-  mcfg.blockDim = dim3(256);
-  mcfg.dynamicSmemBytes = 0;
+  mcfg.blockDim = dim3(pa::merge_threads(D, G));
+  mcfg.dynamicSmemBytes = size_t(p.total_warps) * sizeof(int);
   e = cudaLaunchKernelEx(&mcfg, pa::paged_decode_merge_kernel<T, D, G>, p);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_merge_kernel", e);
   return PA_OK;

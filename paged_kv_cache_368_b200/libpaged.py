@@ -25,7 +25,7 @@ ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
 SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_static",
-           "pa_decode_step_host", "pa_status_string", "pa_version", "pa_last_error")
+           "pa_decode_step_host", "pa_step_inputs_layout", "pa_status_string", "pa_version", "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -62,8 +62,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32, _i32, _i32,
                                      _i64, _i32, _i32, _vp, _vp]
     lib.pa_decode_static.restype = _i32
-    lib.pa_decode_step_host.argtypes = [_vp] * 16 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
-                                                     _vp, _sz, _vp, _vp]
+    lib.pa_step_inputs_layout.argtypes = [_i32, _i32, _i32, _i32, _i32, _c.POINTER(_sz)]
+    lib.pa_step_inputs_layout.restype = _sz
+    lib.pa_decode_step_host.argtypes = [_vp] * 6 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
+                                                    _vp, _sz, _vp, _vp]
     lib.pa_decode_step_host.restype = _i32
     lib.pa_status_string.argtypes = [_i32]
     lib.pa_status_string.restype = _c.c_char_p
@@ -213,31 +215,46 @@ def _host_ptr(t: torch.Tensor, name: str) -> int:
     return t.data_ptr()
 
 
-def decode_step_host(h_q, h_key, h_value, h_slot_mapping, h_block_tables, h_context_lens, h_out,
-                     d_q, d_key, d_value, d_slot_mapping, d_block_tables, d_context_lens, d_out,
-                     k_cache, v_cache, scale: float, max_context_len: Optional[int] = None,
-                     workspace: Optional[torch.Tensor] = None, err_flags: Optional[torch.Tensor] = None,
-                     stream=None) -> torch.Tensor:
-    """One decode step from host tensors (pinned for asynchronous copies):
-    copy the inputs in, append the new K/V, decode, copy the output to
-    ``h_out``.  Returns ``h_out``; valid once the stream is synchronized."""
-    S, H, D = h_q.shape
-    nb, kvh, bs, _ = k_cache.shape
-    mb = h_block_tables.shape[1]
+STEP_INPUTS = ("q", "key", "value", "slot_mapping", "block_tables", "context_lens")
+
+
+def step_inputs_layout(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_blocks_per_seq: int):
+    """(offsets, total bytes) of the packed per-step inputs of ``decode_step_host``."""
+    off = (_sz * 6)()
+    total = load().pa_step_inputs_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq, off)
+    if total == 0:
+        raise LibpagedError(PA_ERR_INVALID, "pa_step_inputs_layout")
+    return dict(zip(STEP_INPUTS, list(off))), int(total)
+
+
+def pack_step_inputs(buf: torch.Tensor, offsets: dict, **tensors) -> torch.Tensor:
+    """Copy host tensors into their slots of a packed uint8 staging buffer."""
+    for name, t in tensors.items():
+        raw = t.contiguous().view(torch.uint8).reshape(-1)
+        buf[offsets[name]: offsets[name] + raw.numel()].copy_(raw)
+    return buf
+
+
+def decode_step_host(h_inputs: torch.Tensor, d_inputs: torch.Tensor, h_out: torch.Tensor, d_out: torch.Tensor,
+                     k_cache: torch.Tensor, v_cache: torch.Tensor, num_heads: int, max_blocks_per_seq: int,
+                     scale: float, max_context_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+                     err_flags: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step from a packed host staging buffer (pinned for
+    asynchronous copies): copy in, append the new K/V, decode, copy the
+    output to ``h_out``.  Returns ``h_out``; valid once the stream is
+    synchronized."""
+    S = h_out.shape[0]
+    nb, kvh, bs, D = k_cache.shape
     if max_context_len is None:
-        max_context_len = mb * bs
+        max_context_len = max_blocks_per_seq * bs
     if workspace is None:
-        workspace = alloc_workspace(S, H, kvh, D, max_context_len, device=k_cache.device)
+        workspace = alloc_workspace(S, num_heads, kvh, D, max_context_len, device=k_cache.device)
     st = load().pa_decode_step_host(
-        _host_ptr(h_q, "h_q"), _host_ptr(h_key, "h_key"), _host_ptr(h_value, "h_value"),
-        _host_ptr(h_slot_mapping, "h_slot_mapping"), _host_ptr(h_block_tables, "h_block_tables"),
-        _host_ptr(h_context_lens, "h_context_lens"), _host_ptr(h_out, "h_out"),
-        _dev_ptr(d_q, "d_q"), _dev_ptr(d_key, "d_key"), _dev_ptr(d_value, "d_value"),
-        _dev_ptr(d_slot_mapping, "d_slot_mapping"), _dev_ptr(d_block_tables, "d_block_tables"),
-        _dev_ptr(d_context_lens, "d_context_lens"), _dev_ptr(d_out, "d_out"),
-        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), S, mb, int(max_context_len), float(scale),
-        H, kvh, D, bs, nb, dtype_code(h_q.dtype), _dev_ptr(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(), _dev_ptr(err_flags, "err_flags"), _stream(stream))
+        _host_ptr(h_inputs, "h_inputs"), _dev_ptr(d_inputs, "d_inputs"), _host_ptr(h_out, "h_out"),
+        _dev_ptr(d_out, "d_out"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), S, max_blocks_per_seq,
+        int(max_context_len), float(scale), num_heads, kvh, D, bs, nb, dtype_code(k_cache.dtype),
+        _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _dev_ptr(err_flags, "err_flags"), _stream(stream))
     if st != PA_OK:
         raise LibpagedError(st, "pa_decode_step_host")
     return h_out

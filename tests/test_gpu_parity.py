@@ -275,25 +275,27 @@ def test_status_codes_through_binding():
 
 
 def test_decode_step_from_host_buffers():
-    """pa_decode_step_host (copies in, append, decode, copy out) gives the same
-    bits as the device-resident calls, and matches the oracle."""
+    """pa_decode_step_host (one packed copy in, append, decode, copy out)
+    gives the same bits as the device-resident calls, and matches the oracle."""
     wl = inputs.random_case(71, num_seqs=6, num_heads=16, num_kv_heads=4, head_dim=128, block_size=16,
                             dtype="bf16", ctx_lo=1, ctx_hi=1500)
     ds = DeviceState(wl, full_pool=True)
     dev_out = ds.step()
     ds2 = DeviceState(wl, full_pool=True)
-    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
-    h_q = pin(wl.q.view(np.int16)).view(torch.bfloat16)
-    h_k = pin(wl.k_new.view(np.int16)).view(torch.bfloat16)
-    h_v = pin(wl.v_new.view(np.int16)).view(torch.bfloat16)
-    h_out = torch.empty_like(h_q).pin_memory()
-    d_q, d_k, d_v = torch.empty_like(ds2.q), torch.empty_like(ds2.k_new), torch.empty_like(ds2.v_new)
-    d_slots, d_tables, d_ctx = torch.empty_like(ds2.slots), torch.empty_like(ds2.tables), torch.empty_like(ds2.ctx)
-    libpaged.decode_step_host(h_q, h_k, h_v, pin(wl.slot_mapping.astype(np.int64)),
-                              pin(wl.block_tables.astype(np.int32)), pin(wl.context_lens.astype(np.int32)), h_out,
-                              d_q, d_k, d_v, d_slots, d_tables, d_ctx, torch.empty_like(ds2.q),
-                              ds2.k_cache, ds2.v_cache, float(wl.scale), max_context_len=wl.max_context_len,
-                              workspace=ds2.ws, err_flags=ds2.err)
+    offs, total = libpaged.step_inputs_layout(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                                              wl.max_blocks_per_seq)
+    assert all(o % 256 == 0 for o in offs.values())
+    h_in = torch.zeros(total, dtype=torch.uint8).pin_memory()
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+    libpaged.pack_step_inputs(h_in, offs, q=t(wl.q), key=t(wl.k_new), value=t(wl.v_new),
+                              slot_mapping=t(wl.slot_mapping.astype(np.int64)),
+                              block_tables=t(wl.block_tables.astype(np.int32)),
+                              context_lens=t(wl.context_lens.astype(np.int32)))
+    d_in = torch.empty(total, dtype=torch.uint8, device="cuda")
+    h_out = torch.empty(ds2.q.shape, dtype=torch.bfloat16).pin_memory()
+    libpaged.decode_step_host(h_in, d_in, h_out, torch.empty_like(ds2.q), ds2.k_cache, ds2.v_cache,
+                              wl.num_heads, wl.max_blocks_per_seq, float(wl.scale),
+                              max_context_len=wl.max_context_len, workspace=ds2.ws, err_flags=ds2.err)
     torch.cuda.synchronize()
     host_out = h_out.view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(host_out, dev_out)
