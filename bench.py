@@ -42,15 +42,20 @@ SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic of one decode launch (dram__bytes_read.sum + dram__bytes_write.sum
-# from an ncu capture), keyed by workload, valid only while the kernel sources
-# hash to `src`.
-NCU_TRAFFIC = {}
+# DRAM traffic of one decode-kernel launch (dram__bytes_read.sum +
+# dram__bytes_write.sum, ncu --set full, profiles/paged_decode_*.md), keyed by
+# workload; reported only while the decode kernel's device sources hash to `src`.
+NCU_TRAFFIC = {
+    "llama7b-mha": {"bytes": 584_963_840 + 4_026_112, "src": "f65eb04587b47385"},
+    "llama3-8b-gqa": {"bytes": 1_148_161_000 + 6_258_176, "src": "f65eb04587b47385"},
+    "long-context-shared-prefix": {"bytes": 1_007_600_000 + 3_718_144, "src": "f65eb04587b47385"},
+}
 
 
 def kernel_source_hash() -> str:
+    """Hash of the decode kernel's device code (the kernel whose traffic is quoted)."""
     h = hashlib.sha256()
-    for f in ("paged_decode.cu", "pa_device.cuh"):
+    for f in ("paged_decode_kernel.cuh", "pa_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_368_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
