@@ -63,7 +63,8 @@ typedef enum {
   PA_ERR_INVALID = 1,     /* null pointer, negative size, bad head ratio, misaligned pointer */
   PA_ERR_UNSUPPORTED = 2, /* head_dim/block_size/group size/num_seqs outside what is compiled */
   PA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
-  PA_ERR_WORKSPACE = 4    /* workspace missing or smaller than pa_decode_workspace_size() */
+  PA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than pa_decode_workspace_size() */
+  PA_ERR_OUT_OF_BLOCKS = 5 /* block manager: not enough free blocks (nothing was changed) */
 } pa_status;
 
 /* Device-side error bits (OR-ed into *err_flags). */
@@ -172,6 +173,98 @@ PA_API pa_status pa_decode_static(void* out, const void* q, const void* k_cache,
                            int num_seqs, int max_context_len, float scale, int num_heads, int num_kv_heads,
                            int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype, int max_ctas,
                            int32_t* err_flags, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write copies inside the paged pools ("【infra之路】10-
+ * PagedAttention 与 KV Cache 管理", section 4.3: shared prefixes and beams share
+ * physical blocks until one writes).  For every pair i, block
+ * block_pairs[2i+1] of k_cache and of v_cache becomes a bit-exact copy of
+ * block block_pairs[2i] (all kv-heads, all rows).  block_pairs: int64 device
+ * array of 2*num_pairs ids.  A block may not be both a source and a
+ * destination in one call.  An id outside [0, num_blocks) skips that pair and
+ * sets PA_ERRF_BLOCK_RANGE.
+ */
+PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_pairs, int64_t num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                         int32_t* err_flags, pa_stream_t stream);
+
+/*
+ * pa_swap_blocks -- move whole blocks between two pools with the same block
+ * size in bytes (block_bytes = num_kv_heads*block_size*head_dim*2), e.g. a
+ * device pool and a pinned host pool (the tutorial's section 4.3 preemption:
+ * swap a request's blocks out to CPU memory and back).  For every pair i,
+ * dst_pool block block_pairs[2i+1] = src_pool block block_pairs[2i].  Call once
+ * for the K pool and once for the V pool.  Each pool, and block_pairs, must be
+ * device memory or pinned (page-locked) host memory; anything else returns
+ * PA_ERR_INVALID without launching.  Out-of-range ids are skipped and flagged
+ * (PA_ERRF_BLOCK_RANGE).
+ */
+PA_API pa_status pa_swap_blocks(const void* src_pool, int64_t src_num_blocks, void* dst_pool, int64_t dst_num_blocks,
+                         int64_t block_bytes, const int64_t* block_pairs, int64_t num_pairs, int32_t* err_flags,
+                         pa_stream_t stream);
+
+/*
+ * Block manager (host memory, not thread-safe): the pool lifecycle of
+ * "PagedAttention：KV Cache 的分页革命" (section Runtime 如何管理 KV Block: a pool
+ * of fixed-size blocks, a free block taken when a step needs space, the page
+ * table updated, blocks returned when a request ends) with the per-request
+ * block tables of the tutorial (section 3.3) and shared, copy-on-write blocks
+ * (section 4.3).  Free blocks are handed out lowest id first.  All functions
+ * return PA_ERR_INVALID for an unknown or duplicate sequence id.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* A manager of blocks 0..num_blocks-1, all free; NULL on bad arguments or no memory. */
+PA_API pa_block_manager* pa_bm_create(int64_t num_blocks, int block_size);
+PA_API void pa_bm_destroy(pa_block_manager* m);
+PA_API int64_t pa_bm_num_free_blocks(const pa_block_manager* m);
+
+/* A new sequence holding num_tokens tokens (positions 0..num_tokens-1). */
+PA_API pa_status pa_bm_add_sequence(pa_block_manager* m, int64_t seq_id, int64_t num_tokens);
+
+/* child shares all of parent's blocks (beam search / shared prefix): the
+ * table is copied, the KV is not. */
+PA_API pa_status pa_bm_fork(pa_block_manager* m, int64_t parent, int64_t child);
+
+/* Room for one more token: returns its slot (block_id*block_size + offset).
+ * A new block is taken when the last one is full; if the last block is shared,
+ * it is replaced by a fresh block and (*cow_src, *cow_dst) name the copy the
+ * caller must make with pa_copy_blocks before writing (else both are -1). */
+PA_API pa_status pa_bm_append_slot(pa_block_manager* m, int64_t seq_id, int64_t* slot, int64_t* cow_src,
+                            int64_t* cow_dst);
+
+/* Release a sequence; blocks no other sequence holds become free. */
+PA_API pa_status pa_bm_free_sequence(pa_block_manager* m, int64_t seq_id);
+
+/* Tokens held by the sequence, or -1 if unknown. */
+PA_API int64_t pa_bm_context_len(const pa_block_manager* m, int64_t seq_id);
+
+/* The sequence's block table into table[0..max_blocks) (-1 after the last
+ * block); *num_blocks gets its length (PA_ERR_INVALID if it exceeds max_blocks). */
+PA_API pa_status pa_bm_block_table(const pa_block_manager* m, int64_t seq_id, int32_t* table, int max_blocks,
+                            int* num_blocks);
+
+/* Free blocks one more token for each listed sequence would take (for
+ * admission control, the tutorial's section 6 scheduler); -1 on bad ids. */
+PA_API int64_t pa_bm_blocks_needed_to_append(const pa_block_manager* m, const int64_t* seq_ids, int num_seqs);
+
+/* One decode step for a batch: appends one token to each sequence and writes
+ * the kernels' inputs (host arrays): block_tables [num_seqs][max_blocks_per_seq],
+ * context_lens [num_seqs] (counting the new token), slot_mapping [num_seqs],
+ * and the copy-on-write pairs cow_pairs [2*num_seqs] (*num_cow_pairs of them).
+ * All-or-nothing: PA_ERR_OUT_OF_BLOCKS or PA_ERR_INVALID leaves the manager
+ * unchanged. */
+PA_API pa_status pa_bm_prepare_decode(pa_block_manager* m, const int64_t* seq_ids, int num_seqs, int max_blocks_per_seq,
+                               int32_t* block_tables, int32_t* context_lens, int64_t* slot_mapping, int64_t* cow_pairs,
+                               int64_t* num_cow_pairs);
+
+/* Move a sequence from manager `from` to manager `to` (e.g. device pool ->
+ * host pool on preemption, and back): fresh blocks are taken in `to`, the
+ * blocks in `from` are released, and pairs[2i], pairs[2i+1] = (block in
+ * `from`, block in `to`) for pa_swap_blocks.  Shared blocks are copied, not
+ * shared, in `to`. */
+PA_API pa_status pa_bm_swap_sequence(pa_block_manager* from, pa_block_manager* to, int64_t seq_id, int64_t* pairs,
+                              int64_t max_pairs, int64_t* num_pairs);
 
 /* Static, human-readable name of a status code. */
 PA_API const char* pa_status_string(pa_status status);

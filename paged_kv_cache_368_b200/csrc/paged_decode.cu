@@ -273,6 +273,7 @@ extern "C" const char* pa_status_string(pa_status status) {
     case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: shape or size outside the compiled set";
     case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA call or kernel launch failed";
     case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing or too small";
+    case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS: not enough free blocks";
   }
   return "unknown pa_status";
 }

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libpaged.so")
 
 PA_F16, PA_BF16 = 0, 1
-PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE, PA_ERR_OUT_OF_BLOCKS = range(6)
 
 ERRF_SLOT_RANGE = 1 << 0
 ERRF_BLOCK_RANGE = 1 << 1
@@ -25,7 +25,10 @@ ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
 SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_static",
-           "pa_decode_step_host", "pa_step_inputs_layout", "pa_status_string", "pa_version", "pa_last_error")
+           "pa_decode_step_host", "pa_step_inputs_layout", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
+           "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slot",
+           "pa_bm_free_sequence", "pa_bm_context_len", "pa_bm_block_table", "pa_bm_blocks_needed_to_append",
+           "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_status_string", "pa_version", "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -258,3 +261,159 @@ def decode_step_host(h_inputs: torch.Tensor, d_inputs: torch.Tensor, h_out: torc
     if st != PA_OK:
         raise LibpagedError(st, "pa_decode_step_host")
     return h_out
+
+
+# ------------------------------------------------------------------ block operations
+
+
+def _setup_block_api(lib):
+    if getattr(lib, "_block_api", False):
+        return lib
+    lib.pa_copy_blocks.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i32, _vp, _vp]
+    lib.pa_copy_blocks.restype = _i32
+    lib.pa_swap_blocks.argtypes = [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _vp, _vp]
+    lib.pa_swap_blocks.restype = _i32
+    P = _vp
+    lib.pa_bm_create.argtypes = [_i64, _i32]
+    lib.pa_bm_create.restype = P
+    lib.pa_bm_destroy.argtypes = [P]
+    lib.pa_bm_destroy.restype = None
+    lib.pa_bm_num_free_blocks.argtypes = [P]
+    lib.pa_bm_num_free_blocks.restype = _i64
+    lib.pa_bm_add_sequence.argtypes = [P, _i64, _i64]
+    lib.pa_bm_fork.argtypes = [P, _i64, _i64]
+    lib.pa_bm_append_slot.argtypes = [P, _i64, _c.POINTER(_i64), _c.POINTER(_i64), _c.POINTER(_i64)]
+    lib.pa_bm_free_sequence.argtypes = [P, _i64]
+    lib.pa_bm_context_len.argtypes = [P, _i64]
+    lib.pa_bm_context_len.restype = _i64
+    lib.pa_bm_block_table.argtypes = [P, _i64, _vp, _i32, _c.POINTER(_i32)]
+    lib.pa_bm_blocks_needed_to_append.argtypes = [P, _vp, _i32]
+    lib.pa_bm_blocks_needed_to_append.restype = _i64
+    lib.pa_bm_prepare_decode.argtypes = [P, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _c.POINTER(_i64)]
+    lib.pa_bm_swap_sequence.argtypes = [P, P, _i64, _vp, _i64, _c.POINTER(_i64)]
+    for f in ("pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slot", "pa_bm_free_sequence", "pa_bm_block_table",
+              "pa_bm_prepare_decode", "pa_bm_swap_sequence"):
+        getattr(lib, f).restype = _i32
+    lib._block_api = True
+    return lib
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_pairs: torch.Tensor,
+                err_flags: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Copy-on-write copies: block ``block_pairs[i, 1]`` of both caches becomes a
+    copy of block ``block_pairs[i, 0]``.  ``block_pairs`` int64 ``[n, 2]`` on the device."""
+    lib = _setup_block_api(load())
+    if block_pairs.dtype != torch.int64:
+        raise ValueError("block_pairs must be int64 [n, 2]")
+    nb, kvh, bs, d = k_cache.shape
+    st = lib.pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+                            _dev_ptr(block_pairs, "block_pairs"), block_pairs.numel() // 2, kvh, d, bs, nb,
+                            dtype_code(k_cache.dtype), _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_copy_blocks")
+
+
+def swap_blocks(src_pool: torch.Tensor, dst_pool: torch.Tensor, block_pairs: torch.Tensor,
+                err_flags: Optional[torch.Tensor] = None, stream=None) -> None:
+    """``dst_pool[block_pairs[i, 1]] = src_pool[block_pairs[i, 0]]`` for pools of
+    equal block size; each pool (and the pairs) on the device or in pinned host memory."""
+    lib = _setup_block_api(load())
+    if src_pool.shape[1:] != dst_pool.shape[1:] or src_pool.dtype != dst_pool.dtype:
+        raise ValueError("pools must have the same block shape and dtype")
+    for t, name in ((src_pool, "src_pool"), (dst_pool, "dst_pool"), (block_pairs, "block_pairs")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"{name} must be on the device or in pinned host memory")
+    block_bytes = src_pool[0].numel() * src_pool.element_size()
+    st = lib.pa_swap_blocks(src_pool.data_ptr(), src_pool.shape[0], dst_pool.data_ptr(), dst_pool.shape[0],
+                            block_bytes, block_pairs.data_ptr(), block_pairs.numel() // 2,
+                            _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_swap_blocks")
+
+
+class BlockManager:
+    """Host block manager (C++ in libpaged): free list (lowest id first),
+    per-sequence block tables, shared copy-on-write blocks, swapping."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        self._lib = _setup_block_api(load())
+        self._h = self._lib.pa_bm_create(num_blocks, block_size)
+        if not self._h:
+            raise LibpagedError(PA_ERR_INVALID, "pa_bm_create")
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h:
+            self._lib.pa_bm_destroy(h)
+
+    def _check(self, st, where):
+        if st != PA_OK:
+            raise LibpagedError(st, where)
+
+    @property
+    def num_free(self) -> int:
+        return int(self._lib.pa_bm_num_free_blocks(self._h))
+
+    def add(self, seq_id: int, num_tokens: int):
+        self._check(self._lib.pa_bm_add_sequence(self._h, seq_id, num_tokens), "pa_bm_add_sequence")
+
+    def fork(self, parent: int, child: int):
+        self._check(self._lib.pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def append_slot(self, seq_id: int):
+        """-> (slot, cow_src, cow_dst)"""
+        slot, src, dst = _i64(), _i64(), _i64()
+        self._check(self._lib.pa_bm_append_slot(self._h, seq_id, _c.byref(slot), _c.byref(src), _c.byref(dst)),
+                    "pa_bm_append_slot")
+        return slot.value, src.value, dst.value
+
+    def free(self, seq_id: int):
+        self._check(self._lib.pa_bm_free_sequence(self._h, seq_id), "pa_bm_free_sequence")
+
+    def context_len(self, seq_id: int) -> int:
+        return int(self._lib.pa_bm_context_len(self._h, seq_id))
+
+    def block_table(self, seq_id: int, max_blocks: int = 1 << 16):
+        import numpy as np
+
+        buf = np.empty(max_blocks, dtype=np.int32)
+        n = _i32()
+        self._check(self._lib.pa_bm_block_table(self._h, seq_id, buf.ctypes.data, max_blocks, _c.byref(n)),
+                    "pa_bm_block_table")
+        return buf[: n.value].tolist()
+
+    def blocks_needed_to_append(self, seq_ids) -> int:
+        import numpy as np
+
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        return int(self._lib.pa_bm_blocks_needed_to_append(self._h, ids.ctypes.data, len(ids)))
+
+    def prepare_decode(self, seq_ids, max_blocks_per_seq: int):
+        """Append one token to each sequence; -> (block_tables, context_lens, slot_mapping, cow_pairs) numpy."""
+        import numpy as np
+
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        tables = np.empty((n, max_blocks_per_seq), dtype=np.int32)
+        ctx = np.empty(n, dtype=np.int32)
+        slots = np.empty(n, dtype=np.int64)
+        cow = np.empty((max(n, 1), 2), dtype=np.int64)
+        ncow = _i64()
+        self._check(self._lib.pa_bm_prepare_decode(self._h, ids.ctypes.data, n, max_blocks_per_seq, tables.ctypes.data,
+                                                   ctx.ctypes.data, slots.ctypes.data, cow.ctypes.data,
+                                                   _c.byref(ncow)), "pa_bm_prepare_decode")
+        return tables, ctx, slots, cow[: ncow.value].copy()
+
+    def swap_to(self, other: "BlockManager", seq_id: int):
+        """Move a sequence into `other`'s pool; -> (n, 2) int64 pairs (block here, block there)."""
+        import numpy as np
+
+        cap = self.num_blocks
+        pairs = np.empty((cap, 2), dtype=np.int64)
+        n = _i64()
+        self._check(self._lib.pa_bm_swap_sequence(self._h, other._h, seq_id, pairs.ctypes.data, cap, _c.byref(n)),
+                    "pa_bm_swap_sequence")
+        return pairs[: n.value].copy()
