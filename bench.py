@@ -448,6 +448,145 @@ def run_ours(args):
     return 0
 
 
+def run_block_ops(args):
+    """Secondary measurement: copy-on-write block copies inside the device pool
+    and swapping blocks to / from pinned host memory, on the LLaMA-7B pool
+    (8400 blocks x 32 kv heads x 16 tokens x 128 x fp16 = 128 KB per block per pool)."""
+    import torch
+
+    from paged_kv_cache_368_b200 import build as pbuild
+    from paged_kv_cache_368_b200 import libpaged
+
+    pbuild.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    nb, kvh, bs, d, npairs = 8400, 32, 16, 128, 1024
+    k = torch.randn((nb, kvh, bs, d), dtype=torch.float16, device=dev)
+    v = torch.randn_like(k)
+    rng = np.random.default_rng(368)
+    ids = rng.permutation(nb)
+    pairs = torch.from_numpy(np.stack([ids[:npairs], ids[npairs:2 * npairs]], 1).astype(np.int64)).to(dev)
+    block_bytes = kvh * bs * d * 2
+    K, W = args.steps, args.warmup
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_src = measured_peak()
+
+    def timed(fn, k_steps):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k_steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / k_steps
+
+    ms = timed(lambda: libpaged.copy_blocks(k, v, pairs), K)
+    moved = 2 * npairs * block_bytes  # K and V pools
+    copy_gbs = 2 * moved / (ms * 1e-3) / 1e9  # read + write, as the STREAM copy counts
+    host = torch.empty((2 * npairs, kvh, bs, d), dtype=torch.float16).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([ids[:npairs], np.arange(npairs)], 1).astype(np.int64)).to(dev)
+    in_pairs = torch.from_numpy(np.stack([np.arange(npairs), ids[npairs:2 * npairs]], 1).astype(np.int64)).to(dev)
+    k_swap = max(3, K // 10)
+    ms_out = timed(lambda: libpaged.swap_blocks(k, host, out_pairs), k_swap)
+    ms_in = timed(lambda: libpaged.swap_blocks(host, k, in_pairs), k_swap)
+    # reference: one contiguous cudaMemcpy of the same bytes in each direction
+    flat_dev = torch.empty(npairs * block_bytes // 2, dtype=torch.float16, device=dev)
+    flat_host = host.view(-1)[: flat_dev.numel()]
+    ms_d2h = timed(lambda: flat_host.copy_(flat_dev, non_blocking=True), k_swap)
+    ms_h2d = timed(lambda: flat_dev.copy_(flat_host, non_blocking=True), k_swap)
+    sw = npairs * block_bytes
+    line = {
+        "metric": "block copy / swap GB/s", "op": "block_ops", "n_gpus": 1, "steps": K, "warmup": W,
+        "config": {"pool": f"{nb} blocks x {kvh} kv heads x {bs} x {d} fp16 ({block_bytes // 1024} KB per block per pool)",
+                   "pairs_per_call": npairs},
+        "copy_blocks": {"us_per_call": ms * 1e3, "bytes_copied": moved, "gbs_read_plus_write": copy_gbs,
+                        "frac_of_copy_peak": copy_gbs / peak, "peak": peak, "peak_source": peak_src},
+        "swap_out_to_pinned_host": {"us_per_call": ms_out * 1e3, "bytes": sw, "gbs": sw / (ms_out * 1e-3) / 1e9,
+                                    "contiguous_memcpy_gbs": sw / (ms_d2h * 1e-3) / 1e9},
+        "swap_in_from_pinned_host": {"us_per_call": ms_in * 1e3, "bytes": sw, "gbs": sw / (ms_in * 1e-3) / 1e9,
+                                     "contiguous_memcpy_gbs": sw / (ms_h2d * 1e-3) / 1e9},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_prefill(args):
+    """Secondary measurement: multi-token causal paged attention (pa_prefill).
+    Workloads: the ops-transformer page's example shape (1 sequence, 32 heads,
+    8192 tokens, head_dim 64, fp16, block_size 16) and a chunked prefill of
+    8 sequences x 1024 new tokens after 1024..3072 cached ones (32 q / 8 kv
+    heads, head_dim 128, bf16)."""
+    import torch
+
+    from paged_kv_cache_368_b200 import build as pbuild
+    from paged_kv_cache_368_b200 import inputs, libpaged
+
+    pbuild.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    K, W = args.steps, args.warmup
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    results = []
+    for name, S, H, KVH, D, dtype, qlen, prefix in (
+            ("ops-transformer example: 1 x 32 heads x 8192 tokens, d 64, fp16", 1, 32, 32, 64, "f16", [8192], [0]),
+            ("chunked prefill: 8 seqs x 1024 new after 1024..3072 cached, 32/8 heads, d 128, bf16", 8, 32, 8, 128,
+             "bf16", [1024] * 8, [1024, 1536, 2048, 2560, 3072, 1024, 2048, 3072])):
+        ctx = [a + b for a, b in zip(qlen, prefix)]
+        wl = inputs.build(name, seed=368, num_seqs=S, num_heads=H, num_kv_heads=KVH, head_dim=D, block_size=16,
+                          dtype=dtype, context_lens=ctx, pool_factor=1.0, poison=False)
+        dt = torch.float16 if dtype == "f16" else torch.bfloat16
+        up = lambda raw: torch.from_numpy(np.ascontiguousarray(raw).view(np.int16).copy()).view(dt).to(dev)  # noqa
+        shape = (wl.num_blocks, KVH, 16, D)
+        kc = torch.zeros(shape, dtype=dt, device=dev)
+        vc = torch.zeros(shape, dtype=dt, device=dev)
+        idx = torch.from_numpy(wl.used).to(dev)
+        kc.index_copy_(0, idx, up(wl.k_blocks))
+        vc.index_copy_(0, idx, up(wl.v_blocks))
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(qlen)]), dtype=torch.int32, device=dev)
+        total = int(sum(qlen))
+        q = torch.randn((total, H, D), dtype=dt, device=dev)
+        out = torch.empty_like(q)
+        tables = torch.from_numpy(wl.block_tables).to(dev)
+        ctx_t = torch.from_numpy(wl.context_lens).to(dev)
+
+        def call():
+            libpaged.prefill(out, q, cu, kc, vc, tables, ctx_t, float(wl.scale), max_q_len=max(qlen),
+                             max_context_len=max(ctx))
+
+        for _ in range(W):
+            call()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            call()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / K
+        # causal FLOPs: row at position p does 2 * 2 * D * (p + 1) per q-head (QK and PV)
+        flops = 0
+        for n, c in zip(qlen, ctx):
+            pos = np.arange(c - n, c, dtype=np.float64)
+            flops += float(4.0 * D * H * (pos + 1).sum())
+        tf = flops / (ms * 1e-3) / 1e12
+        results.append({"workload": name, "us": ms * 1e3, "tflops": tf, "frac_of_bf16_peak": tf / peak,
+                        "kv_bytes_logical": wl.kv_bytes(), "flops": flops})
+    line = {"metric": "pa_prefill causal attention TFLOP/s", "op": "prefill", "n_gpus": 1, "steps": K, "warmup": W,
+            "peak_tflops": peak, "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)",
+            "results": results}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -457,11 +596,18 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (1 = LLaMA-7B-shaped layer)")
     ap.add_argument("--block-size", type=int, default=None, help="block size for workload 3 (LLaMA-13B)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=("step", "block_ops", "prefill"), default="step",
+                    help="step: the decode step (default); block_ops: block copy/swap throughput; "
+                         "prefill: multi-token causal paged attention")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "block_ops":
+        return run_block_ops(args)
+    if args.op == "prefill":
+        return run_prefill(args)
     return run_ours(args)
 
 

@@ -175,6 +175,26 @@ PA_API pa_status pa_decode_static(void* out, const void* q, const void* k_cache,
                            int32_t* err_flags, pa_stream_t stream);
 
 /*
+ * pa_prefill -- multi-token paged attention: several new tokens per sequence
+ * (a prompt, a chunk of one, or speculative tokens) attend causally over the
+ * paged cache (the ops-transformer page's call with a [batch, heads, seq_len,
+ * head_dim] query).  Sequence s owns query rows cu_q_lens[s] ..
+ * cu_q_lens[s+1]-1 of q/out [total_q][num_heads][head_dim]; those n tokens
+ * are the LAST n of its context_lens[s] cached tokens (append them with
+ * pa_reshape_and_cache first), so row i (position ctx-n+i) attends to cached
+ * positions 0..ctx-n+i.  cu_q_lens: int32 device array [num_seqs+1],
+ * non-decreasing, cu_q_lens[0] = 0.  max_q_len bounds the per-sequence n
+ * (sizes the launch).  n > ctx or a context above the bound is clamped and
+ * flags PA_ERRF_CONTEXT.  No workspace.  Same head_dim / block_size support as
+ * pa_decode; num_seqs and num_heads <= 65535.
+ */
+PA_API pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_lens, int total_q, int max_q_len,
+                     const void* k_cache, const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                     const int32_t* context_lens, int num_seqs, int max_context_len, float scale, int num_heads,
+                     int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                     int32_t* err_flags, pa_stream_t stream);
+
+/*
  * pa_copy_blocks -- copy-on-write copies inside the paged pools ("【infra之路】10-
  * PagedAttention 与 KV Cache 管理", section 4.3: shared prefixes and beams share
  * physical blocks until one writes).  For every pair i, block

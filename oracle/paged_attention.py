@@ -135,3 +135,31 @@ def decode_step(q, key, value, k_cache, v_cache, slot_mapping, block_tables, con
     ``(out64, k_cache_after, v_cache_after)``."""
     k2, v2 = reshape_and_cache(key, value, k_cache, v_cache, slot_mapping)
     return decode(q, k2, v2, block_tables, context_lens, scale, dtype), k2, v2
+
+
+def prefill(q, cu_q, k_cache, v_cache, block_tables, context_lens, scale, dtype: str) -> np.ndarray:
+    """Multi-token paged attention (a prompt chunk, or several new tokens):
+    float64 ``[total_q, H, d]``.
+
+    Sequence s owns query rows ``cu_q[s] .. cu_q[s+1]-1``; its ``n = cu_q[s+1]
+    - cu_q[s]`` new tokens are the last n of its ``context_lens[s]`` cached
+    positions (their K/V are already appended), so query row i sits at
+    position ``p = ctx - n + i`` and attends to cached positions ``0..p``
+    (causal).  This is the ops-transformer page's multi-token call (query
+    ``[batch, heads, seq_len, head_dim]`` against the paged cache), each row
+    computed by the section 1.1 formula of the tutorial."""
+    total, H, d = q.shape
+    out = np.zeros((total, H, d))
+    sc = float(np.float32(scale))
+    for s in range(len(context_lens)):
+        lo, hi = int(cu_q[s]), int(cu_q[s + 1])
+        L = int(context_lens[s])
+        n = hi - lo
+        if n == 0 or L == 0:
+            continue
+        k64 = gather(k_cache, block_tables[s], L, dtype)
+        v64 = gather(v_cache, block_tables[s], L, dtype)
+        for i in range(n):
+            p = L - n + i
+            out[lo + i] = attend(widen(q[lo + i], dtype), k64[:, : p + 1], v64[:, : p + 1], sc)
+    return out

@@ -41,10 +41,32 @@
 
 #include "paged_decode_kernel.cuh"
 #include "paged_merge.cuh"
+#include "pa_host.h"
 
 // =============================================================== host side
 
 namespace {
+
+struct WsLayout {
+  size_t header, jobs, ml, o, total;
+};
+
+WsLayout ws_layout(int max_warps, int G, int D) {
+  WsLayout w;
+  w.header = 0;
+  w.jobs = 256;
+  w.ml = w.jobs + (size_t(max_warps) * 16 + 255) / 256 * 256;
+  w.o = w.ml + (size_t(2) * max_warps * G * 8 + 255) / 256 * 256;
+  w.total = w.o + size_t(2) * max_warps * G * D * 4;
+  return w;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+namespace pa {
+thread_local char g_last_error[256] = "no error";
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -63,7 +85,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-constexpr int kMaxDevices = 64;
 
 int device_sms(int dev) {
   static std::atomic<int> cache[kMaxDevices];
@@ -90,26 +111,10 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t nb, int kvh, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-struct WsLayout {
-  size_t header, jobs, ml, o, total;
-};
 
-WsLayout ws_layout(int max_warps, int G, int D) {
-  WsLayout w;
-  w.header = 0;
-  w.jobs = 256;
-  w.ml = w.jobs + (size_t(max_warps) * 16 + 255) / 256 * 256;
-  w.o = w.ml + (size_t(2) * max_warps * G * 8 + 255) / 256 * 256;
-  w.total = w.o + size_t(2) * max_warps * G * D * 4;
-  return w;
-}
 
-inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-}  // namespace
-
-namespace pa {
-thread_local char g_last_error[256] = "no error";
+bool have_tensor_map_encoder() { return encode_fn() != nullptr; }
 
 pa_status fail(pa_status st, const char* what, cudaError_t e) {
   snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, e == cudaSuccess ? "" : cudaGetErrorString(e));
@@ -124,9 +129,9 @@ pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::
                         cudaStream_t stream, int dev) {
   using SH = pa::Shape<D, G>;
   auto kern = pa::paged_decode_kernel<T, D, G>;
-  static std::atomic<int> smem_set[kMaxDevices];
+  static std::atomic<int> smem_set[pa::kMaxDevices];
   const size_t smem = SH::smem_bytes(p.num_seqs);
-  if (dev >= 0 && dev < kMaxDevices && smem_set[dev].load(std::memory_order_relaxed) < (int)smem) {
+  if (dev >= 0 && dev < pa::kMaxDevices && smem_set[dev].load(std::memory_order_relaxed) < (int)smem) {
     // Opt in to the largest dynamic size this kernel can use: the per-block
     // limit minus the kernel's static shared memory.
     int optin = 0;
@@ -187,7 +192,7 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_
   if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  const int sms = device_sms(dev);
+  const int sms = pa::device_sms(dev);
   if (sms <= 0) return 0;
   return ws_layout(sms * pa::warps_for(head_dim, G), G, head_dim).total;
 }
@@ -220,7 +225,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
   if (ce != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaGetDevice", ce);
-  const int sms = device_sms(dev);
+  const int sms = pa::device_sms(dev);
   if (sms <= 0) return pa::fail(PA_ERR_CUDA, "querying the SM count", cudaSuccess);
   const int warps = pa::warps_for(head_dim, G);
   const WsLayout L = ws_layout(sms * warps, G, head_dim);
@@ -230,9 +235,10 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
 
   CUtensorMap km, vm;
-  if (!encode_fn()) return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found", cudaSuccess);
-  if (!make_cache_map(&km, k_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
-      !make_cache_map(&vm, v_cache, num_blocks, num_kv_heads, block_size, head_dim))
+  if (!pa::have_tensor_map_encoder())
+    return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found", cudaSuccess);
+  if (!pa::make_cache_map(&km, k_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
+      !pa::make_cache_map(&vm, v_cache, num_blocks, num_kv_heads, block_size, head_dim))
     return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled rejected the cache layout", cudaSuccess);
 
   pa::DecodeParams p;
