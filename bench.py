@@ -558,20 +558,24 @@ def run_prefill(args):
         tables = torch.from_numpy(wl.block_tables).to(dev)
         ctx_t = torch.from_numpy(wl.context_lens).to(dev)
 
-        def call():
+        def call(legacy=False):
             libpaged.prefill(out, q, cu, kc, vc, tables, ctx_t, float(wl.scale), max_q_len=max(qlen),
-                             max_context_len=max(ctx))
+                             max_context_len=max(ctx), legacy_mma=legacy)
 
-        for _ in range(W):
-            call()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(K):
-            call()
-        e1.record()
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / K
+        def timed(legacy):
+            for _ in range(W):
+                call(legacy)
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(K):
+                call(legacy)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1) / K
+
+        ms = timed(False)
+        ms_mma = timed(True)
         # causal FLOPs: row at position p does 2 * 2 * D * (p + 1) per q-head (QK and PV)
         flops = 0
         for n, c in zip(qlen, ctx):
@@ -579,7 +583,8 @@ def run_prefill(args):
             flops += float(4.0 * D * H * (pos + 1).sum())
         tf = flops / (ms * 1e-3) / 1e12
         results.append({"workload": name, "us": ms * 1e3, "tflops": tf, "frac_of_bf16_peak": tf / peak,
-                        "kv_bytes_logical": wl.kv_bytes(), "flops": flops})
+                        "kv_bytes_logical": wl.kv_bytes(), "flops": flops, "kernel": "tcgen05",
+                        "mma_sync_us": ms_mma * 1e3, "mma_sync_tflops": flops / (ms_mma * 1e-3) / 1e12})
     line = {"metric": "pa_prefill causal attention TFLOP/s", "op": "prefill", "n_gpus": 1, "steps": K, "warmup": W,
             "peak_tflops": peak, "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)",
             "results": results}

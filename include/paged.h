@@ -185,14 +185,24 @@ PA_API pa_status pa_decode_static(void* out, const void* q, const void* k_cache,
  * positions 0..ctx-n+i.  cu_q_lens: int32 device array [num_seqs+1],
  * non-decreasing, cu_q_lens[0] = 0.  max_q_len bounds the per-sequence n
  * (sizes the launch).  n > ctx or a context above the bound is clamped and
- * flags PA_ERRF_CONTEXT.  No workspace.  Same head_dim / block_size support as
- * pa_decode; num_seqs and num_heads <= 65535.
+ * flags PA_ERRF_CONTEXT; offsets outside [0, total_q] skip the sequence and
+ * flag it.  No workspace.  Same head_dim / block_size support as pa_decode;
+ * num_seqs and num_heads <= 65535.  Runs on the tcgen05 tensor cores with
+ * tensor-memory accumulators.
  */
 PA_API pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_lens, int total_q, int max_q_len,
                      const void* k_cache, const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
                      const int32_t* context_lens, int num_seqs, int max_context_len, float scale, int num_heads,
                      int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
                      int32_t* err_flags, pa_stream_t stream);
+
+/* The same operation on the legacy mma.sync tensor-core path (kept as the
+ * reference point the tcgen05 kernel is measured against). */
+PA_API pa_status pa_prefill_mma(void* out, const void* q, const int32_t* cu_q_lens, int total_q, int max_q_len,
+                         const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                         int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int max_context_len,
+                         float scale, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int64_t num_blocks, pa_dtype dtype, int32_t* err_flags, pa_stream_t stream);
 
 /*
  * pa_copy_blocks -- copy-on-write copies inside the paged pools ("【infra之路】10-

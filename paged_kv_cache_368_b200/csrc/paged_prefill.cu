@@ -50,6 +50,7 @@ struct Params {
   int num_kv_heads;
   int block_size;
   int q_tiles;
+  int total_q;
   float scale_log2;
 };
 
@@ -119,7 +120,8 @@ __global__ void __launch_bounds__((kConsumers + 1) * 32, 2)
   const int ctx_raw = __ldg(p.context_lens + s);
   const int ctx = ctx_raw < 0 ? 0 : (ctx_raw > p.ctx_cap ? p.ctx_cap : ctx_raw);
   int n = qb - qa;
-  if (ctx != ctx_raw || n < 0 || n > ctx) {
+  if (qa < 0 || qb > p.total_q) n = 0;  // malformed offsets: touch no row of q or out
+  if (ctx != ctx_raw || n != qb - qa || n > ctx) {
     if (threadIdx.x == 0 && tile == 0 && h == 0) set_err(p.err_flags, PA_ERRF_CONTEXT);
     n = n < 0 ? 0 : (n > ctx ? ctx : n);
   }
@@ -382,7 +384,7 @@ pa_status launch_prefill(const CUtensorMap& km, const CUtensorMap& vm, const pa:
 
 }  // namespace
 
-extern "C" pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_lens, int total_q, int max_q_len,
+extern "C" pa_status pa_prefill_mma(void* out, const void* q, const int32_t* cu_q_lens, int total_q, int max_q_len,
                                 const void* k_cache, const void* v_cache, const int32_t* block_tables,
                                 int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
                                 int max_context_len, float scale, int num_heads, int num_kv_heads, int head_dim,
@@ -426,6 +428,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_le
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;
   p.block_size = block_size;
+  p.total_q = total_q;
   p.q_tiles = (max_q_len + pa::pf::kTileQ - 1) / pa::pf::kTileQ;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -25,7 +25,7 @@ ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
 SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_static",
-           "pa_decode_step_host", "pa_step_inputs_layout", "pa_prefill", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
+           "pa_decode_step_host", "pa_step_inputs_layout", "pa_prefill", "pa_prefill_mma", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
            "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slot",
            "pa_bm_free_sequence", "pa_bm_context_len", "pa_bm_block_table", "pa_bm_blocks_needed_to_append",
            "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_status_string", "pa_version", "pa_last_error")
@@ -70,9 +70,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode_step_host.argtypes = [_vp] * 6 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                                                     _vp, _sz, _vp, _vp]
     lib.pa_decode_step_host.restype = _i32
-    lib.pa_prefill.argtypes = [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32, _i32,
-                               _i32, _i64, _i32, _vp, _vp]
-    lib.pa_prefill.restype = _i32
+    for f in ("pa_prefill", "pa_prefill_mma"):
+        getattr(lib, f).argtypes = [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32,
+                                    _i32, _i32, _i64, _i32, _vp, _vp]
+        getattr(lib, f).restype = _i32
     lib.pa_status_string.argtypes = [_i32]
     lib.pa_status_string.restype = _c.c_char_p
     lib.pa_version.argtypes = []
@@ -425,8 +426,9 @@ class BlockManager:
 def prefill(out: torch.Tensor, q: torch.Tensor, cu_q_lens: torch.Tensor, k_cache: torch.Tensor,
             v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
             max_q_len: int, max_context_len: Optional[int] = None, err_flags: Optional[torch.Tensor] = None,
-            stream=None) -> torch.Tensor:
-    """Causal multi-token paged attention.  ``q``/``out`` ``[total_q, H, D]``;
+            stream=None, legacy_mma: bool = False) -> torch.Tensor:
+    """Causal multi-token paged attention (tcgen05 kernel; ``legacy_mma`` runs
+    the mma.sync kernel instead).  ``q``/``out`` ``[total_q, H, D]``;
     sequence s owns rows ``cu_q_lens[s]..cu_q_lens[s+1]-1``, which are the last
     tokens of its ``context_lens[s]`` cached positions."""
     T, H, D = q.shape
@@ -439,7 +441,8 @@ def prefill(out: torch.Tensor, q: torch.Tensor, cu_q_lens: torch.Tensor, k_cache
     mb = block_tables.shape[1]
     if max_context_len is None:
         max_context_len = mb * bs
-    st = load().pa_prefill(
+    fn = load().pa_prefill_mma if legacy_mma else load().pa_prefill
+    st = fn(
         _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(cu_q_lens, "cu_q_lens"), T, int(max_q_len),
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"), mb,
         _dev_ptr(context_lens, "context_lens"), S, int(max_context_len), float(scale), H, kvh, D, bs, nb,

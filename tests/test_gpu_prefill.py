@@ -32,13 +32,13 @@ def _chunk_case(seed, S, H, KVH, d, bs, dtype, qlens, prefixes, pool_factor=1.5)
     return wl, k, v, cu, q
 
 
-def _run(wl, k, v, cu, q, max_q=None):
+def _run(wl, k, v, cu, q, max_q=None, legacy=False):
     dt = TORCH_DT[wl.dtype]
     out = torch.full((q.shape[0], wl.num_heads, wl.head_dim), float("nan"), dtype=dt, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     libpaged.prefill(out, to_dev(q, wl.dtype), torch.from_numpy(cu).cuda(), to_dev(k, wl.dtype), to_dev(v, wl.dtype),
                      torch.from_numpy(wl.block_tables).cuda(), torch.from_numpy(wl.context_lens).cuda(),
-                     float(wl.scale), max_q_len=int(max_q or np.diff(cu).max()), err_flags=err)
+                     float(wl.scale), max_q_len=int(max_q or np.diff(cu).max()), err_flags=err, legacy_mma=legacy)
     torch.cuda.synchronize()
     return to_raw(out), int(err.item())
 
@@ -46,15 +46,16 @@ def _run(wl, k, v, cu, q, max_q=None):
 SWEEP = [(dt, d, bs, g) for dt in ("f16", "bf16") for d in (64, 128) for bs in (8, 16, 64) for g in (1, 4)]
 
 
+@pytest.mark.parametrize("legacy", [False, True], ids=["tcgen05", "mma"])
 @pytest.mark.parametrize("dtype,d,bs,g", SWEEP, ids=[f"{a}-d{b}-bs{c}-g{e}" for a, b, c, e in SWEEP])
-def test_chunks_match_oracle(dtype, d, bs, g):
+def test_chunks_match_oracle(dtype, d, bs, g, legacy):
     rng = np.random.default_rng(d + bs + g)
     S, kvh = 4, 2
     qlens = rng.integers(1, 150, S)
     prefixes = rng.integers(0, 200, S)
     prefixes[0] = 0  # one whole prompt
     wl, k, v, cu, q = _chunk_case(500 + d + bs * 3 + g, S, kvh * g, kvh, d, bs, dtype, qlens, prefixes)
-    out, err = _run(wl, k, v, cu, q)
+    out, err = _run(wl, k, v, cu, q, legacy=legacy)
     assert err == 0
     ref = oracle.prefill(q, cu, k, v, wl.block_tables, wl.context_lens, wl.scale, dtype)
     assert_close(out, ref, dtype, f"prefill {dtype} d{d} bs{bs} g{g}")
@@ -74,13 +75,14 @@ def test_single_token_chunks_equal_decode_kernel():
     assert_close(to_raw(dec), ref, "bf16", "decode")
 
 
-def test_long_prompt_sampled_rows():
+@pytest.mark.parametrize("legacy", [False, True], ids=["tcgen05", "mma"])
+def test_long_prompt_sampled_rows(legacy):
     """The ops-transformer page's example shape: 1 sequence, 32 heads, 8192
     tokens, head_dim 64, fp16, block_size 16 -- rows checked one by one
     against the oracle's decode of the context that ends at that row."""
     L, H = 8192, 32
     wl, k, v, cu, q = _chunk_case(88, 1, H, H, 64, 16, "f16", [L], [0], pool_factor=1.0)
-    out, err = _run(wl, k, v, cu, q)
+    out, err = _run(wl, k, v, cu, q, legacy=legacy)
     assert err == 0
     assert np.isfinite(oracle.widen(out, "f16")).all()
     kc, vc = k, v
@@ -100,3 +102,14 @@ def test_bad_lengths_are_clamped_and_flagged():
     assert err & libpaged.ERRF_CONTEXT
     ref = oracle.prefill(q[:10], cu[:2], k, v, wl.block_tables[:1], wl.context_lens[:1], wl.scale, "f16")
     assert_close(out[:10], ref, "f16", "first sequence unaffected")
+
+
+def test_malformed_offsets_touch_nothing():
+    wl, k, v, cu, q = _chunk_case(6, 2, 4, 4, 128, 16, "bf16", [20, 30], [5, 0])
+    bad = cu.copy()
+    bad[2] = 10_000  # past total_q
+    out, err = _run(wl, k, v, bad, q, max_q=64)
+    assert err & libpaged.ERRF_CONTEXT
+    ref = oracle.prefill(q[:20], cu[:2], k, v, wl.block_tables[:1], wl.context_lens[:1], wl.scale, "bf16")
+    assert_close(out[:20], ref, "bf16", "first sequence")
+    assert np.all(out[20:] == to_raw(torch.full((1,), float("nan"), dtype=torch.bfloat16))[0])  # untouched
