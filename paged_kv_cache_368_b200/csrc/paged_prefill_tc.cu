@@ -31,12 +31,18 @@
 namespace pa {
 namespace ptc {
 
-constexpr int BM = 128;     // query rows per CTA (MMA M)
-constexpr int BN = 64;      // keys per tile
-constexpr int STAGES = 3;   // K/V ring
-constexpr int kThreads = 256;
+#ifndef PA_PF_BN
+#define PA_PF_BN 64
+#endif
+#ifndef PA_PF_STAGES
+#define PA_PF_STAGES 3
+#endif
+
+constexpr int BM = 128;              // query rows per CTA (MMA M)
+constexpr int BN = PA_PF_BN;         // keys per tile (MMA N of S, K of P.V)
+constexpr int STAGES = PA_PF_STAGES; // K/V ring
 constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr uint32_t kTmemCols = 256;  // S0 [0,64), S1 [64,128), O [128, 128+D)
+
 
 struct Params {
   void* out;
@@ -56,26 +62,41 @@ struct Params {
   float scale_log2;
 };
 
+// Query tiles (softmax warpgroups) per CTA: two share every K/V tile, so the
+// tensor cores alternate between them while each group runs its softmax.
+template <int D>
+struct Groups {
+  static constexpr int kNWG = 2;
+};
+
 template <int D>
 struct Lay {
-  static constexpr int kQ = BM * D * 2;    // [D/64][BM rows][128 B]
+  static constexpr int NWG = Groups<D>::kNWG;
+  static constexpr int kQ = BM * D * 2;    // per group: [D/64][BM rows][128 B]
   static constexpr int kKV = BN * D * 2;   // [D/64][BN rows][128 B]
-  static constexpr int kP = BM * BN * 2;   // [BM rows][128 B]
-  static constexpr int kOffK = kQ;
+  static constexpr int kP = BM * BN * 2;   // per group and buffer: [BN/64][BM rows][128 B]
+  static constexpr int kOffK = NWG * kQ;
   static constexpr int kOffV = kOffK + STAGES * kKV;
   static constexpr int kOffP = kOffV + STAGES * kKV;
-  static constexpr int kOffBar = kOffP + kP;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full, pv_done, mma_done
-  static constexpr int kBars = 1 + 2 * STAGES + 2 + 2 + 3;
+  static constexpr int kOffBar = kOffP + NWG * 2 * kP;  // two P buffers per group
+  // barriers: q_full, kv_full[S], kv_empty[S], and per group s_full[2],
+  // s_free[2], p_full[2], pv_done[2]; then mma_done
+  static constexpr int kBars = 1 + 2 * STAGES + NWG * 8 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kBars * 8 + 16;
+  static constexpr int kThreads = (4 + 4 * NWG) * 32;  // warps 0-3: TMA, MMA, idle, idle
+  static constexpr uint32_t kColsPerGroup = 2 * BN + D;  // S0, S1, O
+  static constexpr uint32_t kTmemCols = NWG * kColsPerGroup <= 256 ? 256u : 512u;
+  static_assert(NWG * kColsPerGroup <= 512, "tensor memory");
+  static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                             const __grid_constant__ CUtensorMap qmap, const Params p) {
   using E = Elem<T>;
   using L = Lay<D>;
+  constexpr int NWG = L::NWG;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -84,11 +105,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + STAGES;
-  uint64_t* s_full = kv_empty + STAGES;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* mma_done = pv_done + 1;
+  // Group g owns bars [8g, 8g+8); every double-buffered barrier is indexed by
+  // the tile's parity so that no waiter can fall two phases behind.
+  uint64_t* grp_bars = kv_empty + STAGES;
+  auto s_full = [&](int g, int b) { return grp_bars + 8 * g + b; };
+  auto s_free = [&](int g, int b) { return grp_bars + 8 * g + 2 + b; };
+  auto p_full = [&](int g, int b) { return grp_bars + 8 * g + 4 + b; };
+  auto pv_done = [&](int g, int b) { return grp_bars + 8 * g + 6 + b; };
+  uint64_t* mma_done = grp_bars + 8 * NWG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,16 +129,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+    for (int g = 0; g < NWG; ++g) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(s_full(g, b), 1);
+        mbar_init(s_free(g, b), 4);
+        mbar_init(pv_done(g, b), 1);
+        mbar_init(p_full(g, b), 4);
+      }
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     fence_barrier_init();
   }
-  if (warp == 1) tc5::tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 1) tc5::tmem_alloc(tmem_slot, L::kTmemCols);
   griddep_wait();
   griddep_launch_dependents();
   tc5::fence_before();
@@ -122,7 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc5::fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Geometry of this sequence and tile.
+  // Geometry: the CTA covers query rows r0 .. r0 + NWG*BM - 1 of the sequence;
+  // group g the BM rows starting at r0 + g*BM.
   const int qa = __ldg(p.cu_q + s), qb = __ldg(p.cu_q + s + 1);
   const int ctx_raw = __ldg(p.context_lens + s);
   const int ctx = ctx_raw < 0 ? 0 : (ctx_raw > p.ctx_cap ? p.ctx_cap : ctx_raw);
@@ -132,12 +159,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && tile == 0 && h == 0) set_err(p.err_flags, PA_ERRF_CONTEXT);
     n = n < 0 ? 0 : (n > ctx ? ctx : n);
   }
-  const int r0 = tile * BM;
-  const bool active = r0 < n;
-  const int rows = active ? min(BM, n - r0) : 0;
-  const int pos0 = ctx - n + r0;
-  const int kend = pos0 + rows;
-  const int ntiles = active ? (kend + BN - 1) / BN : 0;
+  const int r0 = tile * (NWG * BM);
+  auto g_rows = [&](int g) { return max(0, min(BM, n - r0 - g * BM)); };
+  auto g_pos0 = [&](int g) { return ctx - n + r0 + g * BM; };
+  auto g_tiles = [&](int g) { return g_rows(g) > 0 ? (g_pos0(g) + g_rows(g) + BN - 1) / BN : 0; };
+  int ntiles = 0, kend = 0;
+#pragma unroll
+  for (int g = 0; g < NWG; ++g)
+    if (g_rows(g) > 0) {
+      ntiles = g_tiles(g);
+      kend = g_pos0(g) + g_rows(g);
+    }
+  const bool active = ntiles > 0;
   const uint32_t q_s = base, k_s = base + L::kOffK, v_s = base + L::kOffV, p_s = base + L::kOffP;
 
   if (active && warp == 0) {
@@ -146,9 +179,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
     const uint32_t box_bytes = (bs < 16 ? bs : 16) * 128;
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, L::kQ);
+      uint32_t qbytes = 0;
+      for (int g = 0; g < NWG; ++g)
+        if (g_rows(g) > 0) qbytes += L::kQ;
+      mbar_arrive_expect_tx(q_full, qbytes);
+      for (int g = 0; g < NWG; ++g) {
+        if (g_rows(g) == 0) continue;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) tc5::tma_load_3d(q_s + c * (BM * 128), &qmap, q_full, 64 * c, h, qa + r0);
+        for (int c = 0; c < D / 64; ++c)
+          tc5::tma_load_3d(q_s + g * L::kQ + c * (BM * 128), &qmap, q_full, 64 * c, h, qa + r0 + g * BM);
+      }
     }
     const int nchunks = ntiles * (BN / 16);
     bool abort = false;
@@ -170,7 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           b0 = b1 = -1;
         }
       }
-      // one 64-key tile = 4 chunks
       for (int jt = 0; jt < 32 / (BN / 16) && c_base + jt * (BN / 16) < nchunks; ++jt) {
         const int j = c_base / (BN / 16) + jt;
         int bb0[BN / 16], bb1[BN / 16], rr0[BN / 16];
@@ -226,131 +265,164 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int fmt = Elem<T>::kind == PA_BF16 ? 1 : 0;
       constexpr uint32_t id_qk = tc5::f16_idesc(fmt, BM, BN, 0, 0);
       constexpr uint32_t id_pv = tc5::f16_idesc(fmt, BM, D, 0, 1);
+      int gt[NWG];
+#pragma unroll
+      for (int g = 0; g < NWG; ++g) gt[g] = g_tiles(g);
       bool ok = mbar_wait_bounded(q_full, 0, kWaitNs);
-      auto issue_qk = [&](int j) -> bool {
+      auto issue_qk = [&](int g, int j) -> bool {
         const int st = j % STAGES, sb = j & 1;
         if (!mbar_wait_bounded(&kv_full[st], (j / STAGES) & 1, kWaitNs)) return false;
-        if (j >= 2 && !mbar_wait_bounded(&s_free[sb], ((j >> 1) - 1) & 1, kWaitNs)) return false;
+        if (j >= 2 && !mbar_wait_bounded(s_free(g, sb), ((j >> 1) - 1) & 1, kWaitNs)) return false;
         tc5::fence_after();
-        const uint32_t kt = k_s + st * L::kKV;
+        const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
+        const uint32_t sd = tmem + g * L::kColsPerGroup + sb * BN;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t da = tc5::sw128_desc(q_s + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t da = tc5::sw128_desc(qt + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
           const uint64_t db = tc5::sw128_desc(kt + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
-          tc5::mma_ss(tmem + sb * BN, da, db, id_qk, ks > 0);
+          tc5::mma_ss(sd, da, db, id_qk, ks > 0);
         }
-        tc5::commit(&s_full[sb]);
+        tc5::commit(s_full(g, sb));
         return true;
       };
       if (ok) {
         tc5::fence_after();
-        ok = issue_qk(0);
+        for (int g = 0; g < NWG && ok; ++g)
+          if (gt[g] > 0) ok = issue_qk(g, 0);
       }
       for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles && !issue_qk(j + 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait_bounded(p_full, j & 1, kWaitNs)) {
-          ok = false;
-          break;
-        }
-        tc5::fence_after();
+        for (int g = 0; g < NWG && ok; ++g)
+          if (j + 1 < gt[g]) ok = issue_qk(g, j + 1);
         const uint32_t vt = v_s + (j % STAGES) * L::kKV;
+        // On the last tile the group that zeroes its unused V rows goes first.
+        const bool last = j == ntiles - 1;
+        for (int gi = 0; gi < NWG && ok; ++gi) {
+          const int g = last ? NWG - 1 - gi : gi;
+          if (j >= gt[g]) continue;
+          if (!mbar_wait_bounded(p_full(g, j & 1), (j >> 1) & 1, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          tc5::fence_after();
+          const uint32_t pt = p_s + (g * 2 + (j & 1)) * L::kP;
+          const uint32_t od = tmem + g * L::kColsPerGroup + 2 * BN;
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t da = tc5::sw128_desc(p_s + ks * 32, 16, 1024);
-          const uint64_t db = tc5::sw128_desc(vt + ks * (16 * 128), BN * 128, 1024);
-          tc5::mma_ss(tmem + 2 * BN, da, db, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t da = tc5::sw128_desc(pt + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
+            const uint64_t db = tc5::sw128_desc(vt + ks * (16 * 128), BN * 128, 1024);
+            tc5::mma_ss(od, da, db, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          tc5::commit(pv_done(g, j & 1));
         }
-        tc5::commit(pv_done);
-        tc5::commit(&kv_empty[j % STAGES]);
+        if (ok) tc5::commit(&kv_empty[j % STAGES]);
       }
       if (!ok) set_err(p.err_flags, PA_ERRF_TIMEOUT);
       tc5::commit(mma_done);  // lets the CTA free tensor memory once every MMA has finished
     }
   } else if (active && warp >= 4) {
     // ------------------------------------------------------------- softmax
-    const int w = warp - 4;
-    const int r = w * 32 + lane;  // query row of this thread (TMEM lane)
+    const int g = (warp - 4) >> 2;        // query tile (warpgroup) of this warp
+    const int w = warp & 3;               // TMEM lanes 32w..32w+31
+    const int r = w * 32 + lane;          // query row within the group's tile
+    const int rows = g_rows(g), pos0 = g_pos0(g), gtiles = g_tiles(g);
+    int lastg = 0;
+#pragma unroll
+    for (int gg = 0; gg < NWG; ++gg)
+      if (g_rows(gg) > 0) lastg = gg;
+    const int gkend = pos0 + rows;
     const uint32_t lane_off = uint32_t(w * 32) << 16;
-    const int rp = pos0 + r;      // its position
+    const uint32_t s_col = tmem + g * L::kColsPerGroup, o_col = s_col + 2 * BN;
+    const int rp = pos0 + r;  // this row's position
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; j < gtiles; ++j) {
       const int sb = j & 1;
-      const bool got = mbar_wait_bounded(&s_full[sb], (j >> 1) & 1, kWaitNs);
+      const bool got = mbar_wait_bounded(s_full(g, sb), (j >> 1) & 1, kWaitNs);
       if (!__all_sync(kFull, got)) {
         ok = false;
         break;
       }
       tc5::fence_after();
-      uint32_t sr0[32], sr1[32];
-      tc5::ld32(tmem + lane_off + sb * BN, sr0);
-      tc5::ld32(tmem + lane_off + sb * BN + 32, sr1);
+      uint32_t sr[BN / 32][32];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tc5::ld32(s_col + lane_off + sb * BN + c * 32, sr[c]);
       tc5::wait_ld();
       tc5::fence_before();
       __syncwarp();
-      if (lane == 0) tc5::arrive(&s_free[sb]);
+      if (lane == 0) tc5::arrive(s_free(g, sb));
 
       const int key0 = j * BN;
       const bool diag = key0 + BN - 1 > pos0;
       float sv[BN];
-      float mt = -INFINITY;
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
       for (int i = 0; i < BN; ++i) {
-        float v = __uint_as_float(i < 32 ? sr0[i] : sr1[i - 32]) * p.scale_log2;
-        if (diag && (key0 + i > rp || key0 + i >= kend)) v = -INFINITY;
+        float v = __uint_as_float(sr[i >> 5][i & 31]) * p.scale_log2;
+        if (diag && (key0 + i > rp || key0 + i >= gkend)) v = -INFINITY;
         sv[i] = v;
-        mt = fmaxf(mt, v);
+        mx[i & 7] = fmaxf(mx[i & 7], v);
       }
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = fmaxf(m_ref, mt);
       const bool resc = m_new > m_ref + 8.f;  // also true the first time (m_ref = -inf)
-      if (j > 0) {
-        const bool done = mbar_wait_bounded(pv_done, (j - 1) & 1, kWaitNs);
+      // P buffer j&1 is free once the P.V of tile j-2 is done.
+      if (j >= 2) {
+        const bool done = mbar_wait_bounded(pv_done(g, j & 1), ((j >> 1) - 1) & 1, kWaitNs);
+        if (!__all_sync(kFull, done)) {
+          ok = false;
+          break;
+        }
+      }
+      // O may be rescaled only after the P.V of tile j-1 has landed in it.
+      if (j > 0 && __any_sync(kFull, resc)) {
+        const bool done = mbar_wait_bounded(pv_done(g, (j - 1) & 1), ((j - 1) >> 1) & 1, kWaitNs);
         if (!__all_sync(kFull, done)) {
           ok = false;
           break;
         }
         tc5::fence_after();
-        if (__any_sync(kFull, resc)) {  // rescale O rows whose reference max moves
-          const float alpha = resc ? fast_exp2(m_ref - m_new) : 1.f;
+        const float alpha = resc ? fast_exp2(m_ref - m_new) : 1.f;
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tc5::ld32(tmem + lane_off + 2 * BN + cc * 32, o);
-            tc5::wait_ld();
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tc5::ld32(o_col + lane_off + cc * 32, o);
+          tc5::wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tc5::st32(tmem + lane_off + 2 * BN + cc * 32, o);
-          }
-          tc5::wait_st();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tc5::st32(o_col + lane_off + cc * 32, o);
         }
+        tc5::wait_st();
       }
       if (resc) {
         l *= (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - m_new);
         m_ref = m_new;
       }
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;
-      // P row: keys 8c..8c+7 go to 16-byte chunk c, stored at chunk c ^ (r % 8)
-      const uint32_t prow = p_s + r * 128;
+      // P row: keys 8c..8c+7 go to 16-byte chunk c%8 of key block c/8 (64
+      // keys = 128 B per block), stored at chunk (c%8) ^ (r%8)
+      const uint32_t prow = p_s + (g * 2 + (j & 1)) * L::kP + r * 128;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c8 = 0; c8 < BN / 8; ++c8) {
         float pv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = fast_exp2(sv[c8 * 8 + e] - mref);
-          l += pv[e];
-        }
+        for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(sv[c8 * 8 + e] - mref);
+        ls[c8 & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]) + ((pv[4] + pv[5]) + (pv[6] + pv[7]));
         uint4 u;
         u.x = E::pack(pv[0], pv[1]);
         u.y = E::pack(pv[2], pv[3]);
         u.z = E::pack(pv[4], pv[5]);
         u.w = E::pack(pv[6], pv[7]);
-        sts128(prow + ((c8 ^ (r & 7)) << 4), u);
+        sts128(prow + (c8 >> 3) * (BM * 128) + (((c8 & 7) ^ (r & 7)) << 4), u);
       }
-      // V rows at keys >= kend carry zero weight but may hold no data: zero them.
-      if (key0 + BN > kend) {
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // V rows at keys >= the CTA's last visible key carry zero weight for
+      // every row but may hold no data: the last group with rows zeroes them
+      // in the CTA's last tile, and its P.V is issued before the others'.
+      if (g == lastg && key0 + BN > kend) {
         const int vfirst = max(0, kend - key0);
         const uint32_t vt = v_s + (j % STAGES) * L::kKV;
         const int nvec = (BN - vfirst) * (D / 8);
@@ -362,22 +434,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc5::fence_before();
       __syncwarp();
-      if (lane == 0) tc5::arrive(p_full);
+      if (lane == 0) tc5::arrive(p_full(g, j & 1));
     }
-    if (ok) {
-      const bool done = mbar_wait_bounded(pv_done, (ntiles - 1) & 1, kWaitNs);
+    if (ok && gtiles > 0) {
+      const int jl = gtiles - 1;
+      const bool done = mbar_wait_bounded(pv_done(g, jl & 1), (jl >> 1) & 1, kWaitNs);
       ok = __all_sync(kFull, done);
     }
     if (!ok) {
       set_err(p.err_flags, PA_ERRF_TIMEOUT);
-    } else {
+    } else if (gtiles > 0) {
       tc5::fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      T* dst = static_cast<T*>(p.out) + ((int64_t)(qa + r0 + r) * p.num_heads + h) * D;
+      T* dst = static_cast<T*>(p.out) + ((int64_t)(qa + r0 + g * BM + r) * p.num_heads + h) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        tc5::ld32(tmem + lane_off + 2 * BN + cc * 32, o);
+        tc5::ld32(o_col + lane_off + cc * 32, o);
         tc5::wait_ld();
         if (r < rows) {
 #pragma unroll
@@ -400,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (active) mbar_wait_bounded(mma_done, 0, kWaitNs);
     __syncwarp();
     tc5::fence_after();
-    tc5::tmem_free(tmem, kTmemCols);
+    tc5::tmem_free(tmem, L::kTmemCols);
   }
 }
 
@@ -446,7 +519,7 @@ pa_status launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensor
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.q_tiles, p.num_heads, p.num_seqs);
-  cfg.blockDim = dim3(pa::ptc::kThreads);
+  cfg.blockDim = dim3(pa::ptc::Lay<D>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = pdl;
@@ -502,7 +575,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_le
   p.num_kv_heads = num_kv_heads;
   p.block_size = block_size;
   p.total_q = total_q;
-  p.q_tiles = (max_q_len + pa::ptc::BM - 1) / pa::ptc::BM;
+  const int rows_per_cta = pa::ptc::BM * (head_dim == 128 ? pa::ptc::Groups<128>::kNWG : pa::ptc::Groups<64>::kNWG);
+  p.q_tiles = (max_q_len + rows_per_cta - 1) / rows_per_cta;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == PA_F16)

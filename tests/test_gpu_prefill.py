@@ -61,6 +61,20 @@ def test_chunks_match_oracle(dtype, d, bs, g, legacy):
     assert_close(out, ref, dtype, f"prefill {dtype} d{d} bs{bs} g{g}")
 
 
+@pytest.mark.parametrize("legacy", [False, True], ids=["tcgen05", "mma"])
+@pytest.mark.parametrize("dtype,d,bs", [("f16", 64, 8), ("bf16", 128, 16), ("bf16", 64, 32), ("f16", 128, 64)])
+def test_multi_tile_chunks(dtype, d, bs, legacy):
+    """Chunks spanning several 128- and 256-row query tiles with ragged tails,
+    after prefixes that leave the last key tile shared by two query tiles."""
+    qlens = [257, 384, 511, 130, 700, 129]
+    prefixes = [0, 10, 77, 1000, 3, 190]
+    wl, k, v, cu, q = _chunk_case(900 + d + bs, 6, 8, 2, d, bs, dtype, qlens, prefixes)
+    out, err = _run(wl, k, v, cu, q, legacy=legacy)
+    assert err == 0
+    ref = oracle.prefill(q, cu, k, v, wl.block_tables, wl.context_lens, wl.scale, dtype)
+    assert_close(out, ref, dtype, f"prefill multi-tile {dtype} d{d} bs{bs}")
+
+
 def test_single_token_chunks_equal_decode_kernel():
     """With one new token per sequence, prefill is decode: both kernels agree."""
     wl, k, v, cu, q = _chunk_case(77, 6, 8, 2, 128, 16, "bf16", [1] * 6, [5, 100, 700, 33, 1, 2000])
