@@ -187,8 +187,9 @@ PA_API pa_status pa_decode_static(void* out, const void* q, const void* k_cache,
  * (sizes the launch).  n > ctx or a context above the bound is clamped and
  * flags PA_ERRF_CONTEXT; offsets outside [0, total_q] skip the sequence and
  * flag it.  No workspace.  Same head_dim / block_size support as pa_decode;
- * num_seqs and num_heads <= 65535.  Runs on the tcgen05 tensor cores with
- * tensor-memory accumulators.
+ * num_seqs and num_heads <= 65535.  scale must be positive (else
+ * PA_ERR_UNSUPPORTED: the kernel takes row maxima on unscaled scores).  Runs
+ * on the tcgen05 tensor cores with tensor-memory accumulators.
  */
 PA_API pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_lens, int total_q, int max_q_len,
                      const void* k_cache, const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
         int bad = 0;
         if (lane == 0) {
           const int st = j % STAGES;
-          if (j >= STAGES && !mbar_wait_bounded(&kv_empty[st], ((j / STAGES) - 1) & 1, kWaitNs)) {
+          if (j >= STAGES && !tc5::wait(&kv_empty[st], ((j / STAGES) - 1) & 1, kWaitNs)) {
             set_err(p.err_flags, PA_ERRF_TIMEOUT);
             bad = 1;
           } else {
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     // the CTA may exit.
     if (lane == 0) {
       for (int j = max(0, ntiles - STAGES); j < ntiles; ++j)
-        mbar_wait_bounded(&kv_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+        tc5::wait(&kv_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
     }
   } else if (active && warp == 1) {
     // ------------------------------------------------------------- MMA issue
@@ -265,14 +265,11 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       constexpr int fmt = Elem<T>::kind == PA_BF16 ? 1 : 0;
       constexpr uint32_t id_qk = tc5::f16_idesc(fmt, BM, BN, 0, 0);
       constexpr uint32_t id_pv = tc5::f16_idesc(fmt, BM, D, 0, 1);
-      int gt[NWG];
-#pragma unroll
-      for (int g = 0; g < NWG; ++g) gt[g] = g_tiles(g);
-      bool ok = mbar_wait_bounded(q_full, 0, kWaitNs);
+      bool ok = tc5::wait(q_full, 0, kWaitNs);
       auto issue_qk = [&](int g, int j) -> bool {
         const int st = j % STAGES, sb = j & 1;
-        if (!mbar_wait_bounded(&kv_full[st], (j / STAGES) & 1, kWaitNs)) return false;
-        if (j >= 2 && !mbar_wait_bounded(s_free(g, sb), ((j >> 1) - 1) & 1, kWaitNs)) return false;
+        if (!tc5::wait(&kv_full[st], (j / STAGES) & 1, kWaitNs)) return false;
+        if (j >= 2 && !tc5::wait(s_free(g, sb), ((j >> 1) - 1) & 1, kWaitNs)) return false;
         tc5::fence_after();
         const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
         const uint32_t sd = tmem + g * L::kColsPerGroup + sb * BN;
@@ -288,18 +285,18 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       if (ok) {
         tc5::fence_after();
         for (int g = 0; g < NWG && ok; ++g)
-          if (gt[g] > 0) ok = issue_qk(g, 0);
+          if (g_tiles(g) > 0) ok = issue_qk(g, 0);
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         for (int g = 0; g < NWG && ok; ++g)
-          if (j + 1 < gt[g]) ok = issue_qk(g, j + 1);
+          if (j + 1 < g_tiles(g)) ok = issue_qk(g, j + 1);
         const uint32_t vt = v_s + (j % STAGES) * L::kKV;
         // On the last tile the group that zeroes its unused V rows goes first.
         const bool last = j == ntiles - 1;
         for (int gi = 0; gi < NWG && ok; ++gi) {
           const int g = last ? NWG - 1 - gi : gi;
-          if (j >= gt[g]) continue;
-          if (!mbar_wait_bounded(p_full(g, j & 1), (j >> 1) & 1, kWaitNs)) {
+          if (j >= g_tiles(g)) continue;
+          if (!tc5::wait(p_full(g, j & 1), (j >> 1) & 1, kWaitNs)) {
             ok = false;
             break;
           }
@@ -337,7 +334,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     bool ok = true;
     for (int j = 0; j < gtiles; ++j) {
       const int sb = j & 1;
-      const bool got = mbar_wait_bounded(s_full(g, sb), (j >> 1) & 1, kWaitNs);
+      const bool got = tc5::wait(s_full(g, sb), (j >> 1) & 1, kWaitNs);
       if (!__all_sync(kFull, got)) {
         ok = false;
         break;
@@ -352,25 +349,32 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       if (lane == 0) tc5::arrive(s_free(g, sb));
 
       const int key0 = j * BN;
+      // Only tiles that reach past the group's first row need the causal
+      // mask (warp-uniform); keys [0, lim) of the tile are visible to this row.
       const bool diag = key0 + BN - 1 > pos0;
-      float sv[BN];
+      const int lim = diag ? min(rp + 1, gkend) - key0 : BN;
+      float sv[BN];  // raw scores q.k
+#pragma unroll
+      for (int i = 0; i < BN; ++i) sv[i] = __uint_as_float(sr[i >> 5][i & 31]);
+      if (diag) {
+#pragma unroll
+        for (int i = 0; i < BN; ++i) sv[i] = i < lim ? sv[i] : -INFINITY;
+      }
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        float v = __uint_as_float(sr[i >> 5][i & 31]) * p.scale_log2;
-        if (diag && (key0 + i > rp || key0 + i >= gkend)) v = -INFINITY;
-        sv[i] = v;
-        mx[i & 7] = fmaxf(mx[i & 7], v);
-      }
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int i = 0; i < BN; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = tc5::max3(mx[k], sv[i + k], sv[i + 8 + k]);
+      const float rmax = tc5::max3(tc5::max3(mx[0], mx[1], mx[2]), tc5::max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      // the scale is positive (checked on the host), so it commutes with the max
+      const float mt = rmax == -INFINITY ? -INFINITY : rmax * p.scale_log2;
       const float m_new = fmaxf(m_ref, mt);
       const bool resc = m_new > m_ref + 8.f;  // also true the first time (m_ref = -inf)
       // P buffer j&1 is free once the P.V of tile j-2 is done.
       if (j >= 2) {
-        const bool done = mbar_wait_bounded(pv_done(g, j & 1), ((j >> 1) - 1) & 1, kWaitNs);
+        const bool done = tc5::wait(pv_done(g, j & 1), ((j >> 1) - 1) & 1, kWaitNs);
         if (!__all_sync(kFull, done)) {
           ok = false;
           break;
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       }
       // O may be rescaled only after the P.V of tile j-1 has landed in it.
       if (j > 0 && __any_sync(kFull, resc)) {
-        const bool done = mbar_wait_bounded(pv_done(g, (j - 1) & 1), ((j - 1) >> 1) & 1, kWaitNs);
+        const bool done = tc5::wait(pv_done(g, (j - 1) & 1), ((j - 1) >> 1) & 1, kWaitNs);
         if (!__all_sync(kFull, done)) {
           ok = false;
           break;
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       for (int c8 = 0; c8 < BN / 8; ++c8) {
         float pv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(sv[c8 * 8 + e] - mref);
+        for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(fmaf(sv[c8 * 8 + e], p.scale_log2, -mref));
         ls[c8 & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]) + ((pv[4] + pv[5]) + (pv[6] + pv[7]));
         uint4 u;
         u.x = E::pack(pv[0], pv[1]);
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     }
     if (ok && gtiles > 0) {
       const int jl = gtiles - 1;
-      const bool done = mbar_wait_bounded(pv_done(g, jl & 1), (jl >> 1) & 1, kWaitNs);
+      const bool done = tc5::wait(pv_done(g, jl & 1), (jl >> 1) & 1, kWaitNs);
       ok = __all_sync(kFull, done);
     }
     if (!ok) {
@@ -470,7 +474,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
   tc5::fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (active) mbar_wait_bounded(mma_done, 0, kWaitNs);
+    if (active) tc5::wait(mma_done, 0, kWaitNs);
     __syncwarp();
     tc5::fence_after();
     tc5::tmem_free(tmem, L::kTmemCols);
@@ -544,6 +548,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_le
   if (max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0) return PA_ERR_INVALID;
   if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID;
   if (!std::isfinite(scale)) return PA_ERR_INVALID;
+  if (!(scale > 0.f)) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64) return PA_ERR_UNSUPPORTED;
   if (num_seqs > 65535 || num_heads > 65535) return PA_ERR_UNSUPPORTED;

@@ -97,6 +97,39 @@ __device__ __forceinline__ void arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// max(a, b, c) in one instruction (three-input form, sm_100 and later).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// One mbarrier probe that lets the hardware suspend the thread for up to
+// `hint_ns` while the phase is still open, so waiting warps take no issue slots.
+__device__ __forceinline__ bool try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, giving up after `limit_ns`
+// (the caller records the timeout and unwinds).
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  constexpr uint32_t kHintNs = 1u << 20;  // about 1 ms per probe
+  if (try_wait_suspend(bar, parity, kHintNs)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (try_wait_suspend(bar, parity, kHintNs)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // 4-D tiled TMA load without an L2 policy.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
                                             int c3) {

@@ -92,6 +92,35 @@ def test_reshape_host_checks(lib):
     assert call(T=0) == libpaged.PA_OK
 
 
+@pytest.mark.parametrize("entry", ["pa_prefill", "pa_prefill_mma"])
+def test_prefill_host_checks(lib, entry):
+    f = getattr(lib, entry)
+    I, U = libpaged.PA_ERR_INVALID, libpaged.PA_ERR_UNSUPPORTED
+    ok = dict(out=16, q=16, cu=16, T=40, maxq=20, k=16, v=16, tables=16, mb=4, ctx=16, S=2, maxctx=64, scale=0.1,
+              H=4, KVH=2, D=64, BS=16, NB=8, dt=1)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["out"], a["q"], a["cu"], a["T"], a["maxq"], a["k"], a["v"], a["tables"], a["mb"], a["ctx"],
+                 a["S"], a["maxctx"], a["scale"], a["H"], a["KVH"], a["D"], a["BS"], a["NB"], a["dt"], None, None)
+
+    assert call(H=6, KVH=4) == I
+    assert call(T=-1) == I
+    assert call(mb=0) == I
+    assert call(dt=3) == I
+    assert call(scale=float("nan")) == I
+    assert call(D=256) == U
+    assert call(BS=4) == U
+    assert call(S=70000) == U
+    assert call(out=None) == I
+    assert call(cu=2) == I  # misaligned int32
+    assert call(S=0) == libpaged.PA_OK
+    if entry == "pa_prefill":
+        assert call(scale=0.0) == U  # row maxima are taken on unscaled scores
+        assert call(scale=-0.1) == U
+
+
 def test_workspace_size_rejects_bad_shapes(lib):
     assert lib.pa_decode_workspace_size(4, 6, 4, 128, 100) == 0
     assert lib.pa_decode_workspace_size(4, 32, 2, 128, 100) == 0  # group of 16
