@@ -31,16 +31,9 @@
 namespace pa {
 namespace ptc {
 
-#ifndef PA_PF_BN
-#define PA_PF_BN 64
-#endif
-#ifndef PA_PF_STAGES
-#define PA_PF_STAGES 3
-#endif
-
-constexpr int BM = 128;              // query rows per CTA (MMA M)
-constexpr int BN = PA_PF_BN;         // keys per tile (MMA N of S, K of P.V)
-constexpr int STAGES = PA_PF_STAGES; // K/V ring
+constexpr int BM = 128;  // query rows per softmax group (MMA M)
+constexpr int BN = 64;   // keys per tile (MMA N of S, K of P.V)
+constexpr int kGroups = 2;  // query tiles (softmax warpgroups) per CTA sharing each K/V tile
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 
@@ -62,29 +55,23 @@ struct Params {
   float scale_log2;
 };
 
-// Query tiles (softmax warpgroups) per CTA: two share every K/V tile, so the
-// tensor cores alternate between them while each group runs its softmax.
-template <int D>
-struct Groups {
-  static constexpr int kNWG = 2;
-};
-
 template <int D>
 struct Lay {
-  static constexpr int NWG = Groups<D>::kNWG;
-  static constexpr int kQ = BM * D * 2;    // per group: [D/64][BM rows][128 B]
-  static constexpr int kKV = BN * D * 2;   // [D/64][BN rows][128 B]
-  static constexpr int kP = BM * BN * 2;   // per group and buffer: [BN/64][BM rows][128 B]
+  static constexpr int NWG = kGroups;
+  static constexpr int STAGES = D == 128 ? 5 : 8;  // K/V ring depth (tiles in flight)
+  static constexpr int kQ = BM * D * 2;   // per group: [D/64][BM rows][128 B]
+  static constexpr int kKV = BN * D * 2;  // one K or V tile: [D/64][BN rows][128 B]
   static constexpr int kOffK = NWG * kQ;
   static constexpr int kOffV = kOffK + STAGES * kKV;
-  static constexpr int kOffP = kOffV + STAGES * kKV;
-  static constexpr int kOffBar = kOffP + NWG * 2 * kP;  // two P buffers per group
-  // barriers: q_full, kv_full[S], kv_empty[S], and per group s_full[2],
-  // s_free[2], p_full[2], pv_done[2]; then mma_done
-  static constexpr int kBars = 1 + 2 * STAGES + NWG * 8 + 1;
+  static constexpr int kOffBar = kOffV + STAGES * kKV;
+  // barriers: q_full, k_full[S], v_full[S], kv_empty[S]; per group s_full[2],
+  // p_full[2], pv_done[2]; mma_done
+  static constexpr int kBars = 1 + 3 * STAGES + NWG * 6 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kBars * 8 + 16;
   static constexpr int kThreads = (4 + 4 * NWG) * 32;  // warps 0-3: TMA, MMA, idle, idle
-  static constexpr uint32_t kColsPerGroup = 2 * BN + D;  // S0, S1, O
+  // Tensor memory per group: S0 | S1 | O.  P of tile j (16-bit, two per
+  // column) overwrites the front of S(j & 1) once the softmax has read it.
+  static constexpr uint32_t kColsPerGroup = 2 * BN + D;
   static constexpr uint32_t kTmemCols = NWG * kColsPerGroup <= 256 ? 256u : 512u;
   static_assert(NWG * kColsPerGroup <= 512, "tensor memory");
   static_assert(kSmem <= 232448, "shared memory per CTA");
@@ -96,23 +83,23 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
                             const __grid_constant__ CUtensorMap qmap, const Params p) {
   using E = Elem<T>;
   using L = Lay<D>;
-  constexpr int NWG = L::NWG;
+  constexpr int NWG = L::NWG, STAGES = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + STAGES;
-  // Group g owns bars [8g, 8g+8); every double-buffered barrier is indexed by
-  // the tile's parity so that no waiter can fall two phases behind.
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + STAGES;
+  uint64_t* kv_empty = v_full + STAGES;
+  // Group g owns bars [6g, 6g+6); double-buffered barriers are indexed by the
+  // tile's parity, so no waiter can fall two phases behind.
   uint64_t* grp_bars = kv_empty + STAGES;
-  auto s_full = [&](int g, int b) { return grp_bars + 8 * g + b; };
-  auto s_free = [&](int g, int b) { return grp_bars + 8 * g + 2 + b; };
-  auto p_full = [&](int g, int b) { return grp_bars + 8 * g + 4 + b; };
-  auto pv_done = [&](int g, int b) { return grp_bars + 8 * g + 6 + b; };
-  uint64_t* mma_done = grp_bars + 8 * NWG;
+  auto s_full = [&](int g, int b) { return grp_bars + 6 * g + b; };
+  auto p_full = [&](int g, int b) { return grp_bars + 6 * g + 2 + b; };
+  auto pv_done = [&](int g, int b) { return grp_bars + 6 * g + 4 + b; };
+  uint64_t* mma_done = grp_bars + 6 * NWG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,15 +113,15 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     prefetch_tensormap(&qmap);
     mbar_init(q_full, 1);
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&kv_full[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
     for (int g = 0; g < NWG; ++g) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(s_full(g, b), 1);
-        mbar_init(s_free(g, b), 4);
-        mbar_init(pv_done(g, b), 1);
         mbar_init(p_full(g, b), 4);
+        mbar_init(pv_done(g, b), 1);
       }
     }
     mbar_init(mma_done, 1);
@@ -163,15 +150,16 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
   auto g_rows = [&](int g) { return max(0, min(BM, n - r0 - g * BM)); };
   auto g_pos0 = [&](int g) { return ctx - n + r0 + g * BM; };
   auto g_tiles = [&](int g) { return g_rows(g) > 0 ? (g_pos0(g) + g_rows(g) + BN - 1) / BN : 0; };
-  int ntiles = 0, kend = 0;
+  int ntiles = 0, kend = 0, lastg = 0;
 #pragma unroll
   for (int g = 0; g < NWG; ++g)
     if (g_rows(g) > 0) {
       ntiles = g_tiles(g);
       kend = g_pos0(g) + g_rows(g);
+      lastg = g;
     }
   const bool active = ntiles > 0;
-  const uint32_t q_s = base, k_s = base + L::kOffK, v_s = base + L::kOffV, p_s = base + L::kOffP;
+  const uint32_t q_s = base, k_s = base + L::kOffK, v_s = base + L::kOffV;
 
   if (active && warp == 0) {
     // ------------------------------------------------------------- producer
@@ -226,22 +214,25 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
             set_err(p.err_flags, PA_ERRF_TIMEOUT);
             bad = 1;
           } else {
-            uint32_t bytes = 0;
+            uint32_t bytes = 0;  // per pool
 #pragma unroll
             for (int q = 0; q < BN / 16; ++q)
-              bytes += (bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1)) * (D / 64) * box_bytes * 2;
-            mbar_arrive_expect_tx(&kv_full[st], bytes);
-            const uint32_t kt = k_s + st * L::kKV, vt = v_s + st * L::kKV;
+              bytes += (bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1)) * (D / 64) * box_bytes;
+            // K first: the score MMA needs only K; V is consumed later.
+            for (int kv = 0; kv < 2; ++kv) {
+              uint64_t* full = kv == 0 ? &k_full[st] : &v_full[st];
+              const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
+              const uint32_t dst = (kv == 0 ? k_s : v_s) + st * L::kKV;
+              mbar_arrive_expect_tx(full, bytes);
 #pragma unroll
-            for (int q = 0; q < BN / 16; ++q) {
-              const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
-              for (int b = 0; b < nb; ++b) {
-                const int phys = b == 0 ? bb0[q] : bb1[q];
+              for (int q = 0; q < BN / 16; ++q) {
+                const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
+                for (int b = 0; b < nb; ++b) {
+                  const int phys = b == 0 ? bb0[q] : bb1[q];
 #pragma unroll
-                for (int cq = 0; cq < D / 64; ++cq) {
-                  const uint32_t off = cq * (BN * 128) + q * 2048 + b * 1024;
-                  tc5::tma_load_4d(kt + off, &kmap, &kv_full[st], 64 * cq, rr0[q], kvh, phys);
-                  tc5::tma_load_4d(vt + off, &vmap, &kv_full[st], 64 * cq, rr0[q], kvh, phys);
+                  for (int cq = 0; cq < D / 64; ++cq)
+                    tc5::tma_load_4d(dst + cq * (BN * 128) + q * 2048 + b * 1024, map, full, 64 * cq, rr0[q], kvh,
+                                     phys);
                 }
               }
             }
@@ -256,85 +247,91 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     // The last tiles' copies have landed (always, on the normal path) before
     // the CTA may exit.
     if (lane == 0) {
-      for (int j = max(0, ntiles - STAGES); j < ntiles; ++j)
-        tc5::wait(&kv_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+      for (int j = max(0, ntiles - STAGES); j < ntiles; ++j) {
+        tc5::wait(&k_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+        tc5::wait(&v_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+      }
     }
   } else if (active && warp == 1) {
     // ------------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      constexpr int fmt = Elem<T>::kind == PA_BF16 ? 1 : 0;
-      constexpr uint32_t id_qk = tc5::f16_idesc(fmt, BM, BN, 0, 0);
-      constexpr uint32_t id_pv = tc5::f16_idesc(fmt, BM, D, 0, 1);
-      bool ok = tc5::wait(q_full, 0, kWaitNs);
-      auto issue_qk = [&](int g, int j) -> bool {
-        const int st = j % STAGES, sb = j & 1;
-        if (!tc5::wait(&kv_full[st], (j / STAGES) & 1, kWaitNs)) return false;
-        if (j >= 2 && !tc5::wait(s_free(g, sb), ((j >> 1) - 1) & 1, kWaitNs)) return false;
-        tc5::fence_after();
-        const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
-        const uint32_t sd = tmem + g * L::kColsPerGroup + sb * BN;
+    // The whole warp follows the schedule (so descriptors stay warp-uniform);
+    // one elected lane issues every MMA and commit.  Per tile j and group g:
+    // P.V of tile j, then the scores of tile j+2 into the S buffer that P
+    // occupied (tensor-core operations of one thread run in issue order).
+    constexpr int fmt = Elem<T>::kind == PA_BF16 ? 1 : 0;
+    constexpr uint32_t id_qk = tc5::f16_idesc(fmt, BM, BN, 0, 0);
+    constexpr uint32_t id_pv = tc5::f16_idesc(fmt, BM, D, 0, 1);
+    const uint32_t leader = tc5::elect_one();
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool got = tc5::wait(bar, parity, kWaitNs);
+      return __all_sync(kFull, got);
+    };
+    auto issue_qk = [&](int g, int j) -> bool {  // S(g, j&1) = Q_g K_j^T
+      const int st = j % STAGES;
+      if (!wait_all(&k_full[st], (j / STAGES) & 1)) return false;
+      tc5::fence_after();
+      const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
+      const uint32_t sd = tmem + g * L::kColsPerGroup + (j & 1) * BN;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t da = tc5::sw128_desc(qt + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t db = tc5::sw128_desc(kt + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
-          tc5::mma_ss(sd, da, db, id_qk, ks > 0);
-        }
-        tc5::commit(s_full(g, sb));
-        return true;
-      };
-      if (ok) {
-        tc5::fence_after();
-        for (int g = 0; g < NWG && ok; ++g)
-          if (g_tiles(g) > 0) ok = issue_qk(g, 0);
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t da = tc5::sw128_desc(qt + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
+        const uint64_t db = tc5::sw128_desc(kt + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
+        tc5::mma_ss_if(leader, sd, da, db, id_qk, ks > 0);
       }
-      for (int j = 0; ok && j < ntiles; ++j) {
-        for (int g = 0; g < NWG && ok; ++g)
-          if (j + 1 < g_tiles(g)) ok = issue_qk(g, j + 1);
-        const uint32_t vt = v_s + (j % STAGES) * L::kKV;
-        // On the last tile the group that zeroes its unused V rows goes first.
-        const bool last = j == ntiles - 1;
-        for (int gi = 0; gi < NWG && ok; ++gi) {
-          const int g = last ? NWG - 1 - gi : gi;
-          if (j >= g_tiles(g)) continue;
-          if (!tc5::wait(p_full(g, j & 1), (j >> 1) & 1, kWaitNs)) {
-            ok = false;
-            break;
-          }
-          tc5::fence_after();
-          const uint32_t pt = p_s + (g * 2 + (j & 1)) * L::kP;
-          const uint32_t od = tmem + g * L::kColsPerGroup + 2 * BN;
+      tc5::commit_if(leader, s_full(g, j & 1));
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](int g, int j) -> bool {  // O_g += P(g, j) V_j, P from tensor memory
+      const int st = j % STAGES;
+      if (!wait_all(&v_full[st], (j / STAGES) & 1)) return false;
+      if (!wait_all(p_full(g, j & 1), (j >> 1) & 1)) return false;
+      tc5::fence_after();
+      const uint32_t vt = v_s + st * L::kKV;
+      const uint32_t pa = tmem + g * L::kColsPerGroup + (j & 1) * BN;
+      const uint32_t od = tmem + g * L::kColsPerGroup + 2 * BN;
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t da = tc5::sw128_desc(pt + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
-            const uint64_t db = tc5::sw128_desc(vt + ks * (16 * 128), BN * 128, 1024);
-            tc5::mma_ss(od, da, db, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          tc5::commit(pv_done(g, j & 1));
-        }
-        if (ok) tc5::commit(&kv_empty[j % STAGES]);
+      for (int ks = 0; ks < BN / 16; ++ks) {
+        const uint64_t db = tc5::sw128_desc(vt + ks * (16 * 128), BN * 128, 1024);
+        tc5::mma_ts_if(leader, od, pa + ks * 8, db, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
       }
-      if (!ok) set_err(p.err_flags, PA_ERRF_TIMEOUT);
-      tc5::commit(mma_done);  // lets the CTA free tensor memory once every MMA has finished
+      tc5::commit_if(leader, pv_done(g, j & 1));
+      __syncwarp();
+      return true;
+    };
+    bool ok = wait_all(q_full, 0);
+    if (ok) tc5::fence_after();
+    for (int j = 0; j < 2 && ok; ++j)
+      for (int g = 0; g < NWG && ok; ++g)
+        if (j < g_tiles(g)) ok = issue_qk(g, j);
+    for (int j = 0; ok && j < ntiles; ++j) {
+      // On the CTA's last tile the group that zeroes the unused V rows goes first.
+      const bool last = j == ntiles - 1;
+      for (int gi = 0; gi < NWG && ok; ++gi) {
+        const int g = last ? NWG - 1 - gi : gi;
+        const bool uses = j < g_tiles(g);
+        if (uses) ok = issue_pv(g, j);
+        if (ok && gi == NWG - 1) tc5::commit_if(leader, &kv_empty[j % STAGES]);  // every P.V of tile j issued
+        if (ok && uses && j + 2 < g_tiles(g)) ok = issue_qk(g, j + 2);
+      }
     }
+    if (!ok && leader) set_err(p.err_flags, PA_ERRF_TIMEOUT);
+    tc5::commit_if(leader, mma_done);  // lets the CTA free tensor memory once every MMA has finished
   } else if (active && warp >= 4) {
     // ------------------------------------------------------------- softmax
-    const int g = (warp - 4) >> 2;        // query tile (warpgroup) of this warp
-    const int w = warp & 3;               // TMEM lanes 32w..32w+31
-    const int r = w * 32 + lane;          // query row within the group's tile
+    const int g = (warp - 4) >> 2;  // query tile (warpgroup) of this warp
+    const int w = warp & 3;         // tensor-memory lanes 32w..32w+31
+    const int r = w * 32 + lane;    // query row within the group's tile
     const int rows = g_rows(g), pos0 = g_pos0(g), gtiles = g_tiles(g);
-    int lastg = 0;
-#pragma unroll
-    for (int gg = 0; gg < NWG; ++gg)
-      if (g_rows(gg) > 0) lastg = gg;
     const int gkend = pos0 + rows;
     const uint32_t lane_off = uint32_t(w * 32) << 16;
-    const uint32_t s_col = tmem + g * L::kColsPerGroup, o_col = s_col + 2 * BN;
+    const uint32_t s_col = tmem + g * L::kColsPerGroup + lane_off, o_col = s_col + 2 * BN;
     const int rp = pos0 + r;  // this row's position
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < gtiles; ++j) {
-      const int sb = j & 1;
-      const bool got = tc5::wait(s_full(g, sb), (j >> 1) & 1, kWaitNs);
+      const uint32_t sj = s_col + (j & 1) * BN;
+      const bool got = tc5::wait(s_full(g, j & 1), (j >> 1) & 1, kWaitNs);
       if (!__all_sync(kFull, got)) {
         ok = false;
         break;
@@ -342,11 +339,8 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       tc5::fence_after();
       uint32_t sr[BN / 32][32];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tc5::ld32(s_col + lane_off + sb * BN + c * 32, sr[c]);
+      for (int c = 0; c < BN / 32; ++c) tc5::ld32(sj + c * 32, sr[c]);
       tc5::wait_ld();
-      tc5::fence_before();
-      __syncwarp();
-      if (lane == 0) tc5::arrive(s_free(g, sb));
 
       const int key0 = j * BN;
       // Only tiles that reach past the group's first row need the causal
@@ -372,14 +366,6 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       const float mt = rmax == -INFINITY ? -INFINITY : rmax * p.scale_log2;
       const float m_new = fmaxf(m_ref, mt);
       const bool resc = m_new > m_ref + 8.f;  // also true the first time (m_ref = -inf)
-      // P buffer j&1 is free once the P.V of tile j-2 is done.
-      if (j >= 2) {
-        const bool done = tc5::wait(pv_done(g, j & 1), ((j >> 1) - 1) & 1, kWaitNs);
-        if (!__all_sync(kFull, done)) {
-          ok = false;
-          break;
-        }
-      }
       // O may be rescaled only after the P.V of tile j-1 has landed in it.
       if (j > 0 && __any_sync(kFull, resc)) {
         const bool done = tc5::wait(pv_done(g, (j - 1) & 1), ((j - 1) >> 1) & 1, kWaitNs);
@@ -392,22 +378,21 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
-          tc5::ld32(o_col + lane_off + cc * 32, o);
+          tc5::ld32(o_col + cc * 32, o);
           tc5::wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tc5::st32(o_col + lane_off + cc * 32, o);
+          tc5::st32(o_col + cc * 32, o);
         }
-        tc5::wait_st();
       }
       if (resc) {
         l *= (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - m_new);
         m_ref = m_new;
       }
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;
-      // P row: keys 8c..8c+7 go to 16-byte chunk c%8 of key block c/8 (64
-      // keys = 128 B per block), stored at chunk (c%8) ^ (r%8)
-      const uint32_t prow = p_s + (g * 2 + (j & 1)) * L::kP + r * 128;
+      // P row, 16-bit, two keys per tensor-memory column, into the front of
+      // this tile's S buffer (already read).
+      uint32_t pk[BN / 2];
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c8 = 0; c8 < BN / 8; ++c8) {
@@ -415,18 +400,21 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(fmaf(sv[c8 * 8 + e], p.scale_log2, -mref));
         ls[c8 & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]) + ((pv[4] + pv[5]) + (pv[6] + pv[7]));
-        uint4 u;
-        u.x = E::pack(pv[0], pv[1]);
-        u.y = E::pack(pv[2], pv[3]);
-        u.z = E::pack(pv[4], pv[5]);
-        u.w = E::pack(pv[6], pv[7]);
-        sts128(prow + (c8 >> 3) * (BM * 128) + (((c8 & 7) ^ (r & 7)) << 4), u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pk[c8 * 4 + e] = E::pack(pv[2 * e], pv[2 * e + 1]);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tc5::st32(sj, pk);
       // V rows at keys >= the CTA's last visible key carry zero weight for
       // every row but may hold no data: the last group with rows zeroes them
-      // in the CTA's last tile, and its P.V is issued before the others'.
+      // in the CTA's last tile (once its copy has landed), and its P.V is
+      // issued before the others'.
       if (g == lastg && key0 + BN > kend) {
+        const bool vin = tc5::wait(&v_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+        if (!__all_sync(kFull, vin)) {
+          ok = false;
+          break;
+        }
         const int vfirst = max(0, kend - key0);
         const uint32_t vt = v_s + (j % STAGES) * L::kKV;
         const int nvec = (BN - vfirst) * (D / 8);
@@ -434,8 +422,9 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
           const int vr = vfirst + i / (D / 8), c16 = i % (D / 8);
           sts128(vt + (c16 >> 3) * (BN * 128) + vr * 128 + (((c16 & 7) ^ (vr & 7)) << 4), make_uint4(0, 0, 0, 0));
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      tc5::wait_st();
       tc5::fence_before();
       __syncwarp();
       if (lane == 0) tc5::arrive(p_full(g, j & 1));
@@ -454,7 +443,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        tc5::ld32(o_col + lane_off + cc * 32, o);
+        tc5::ld32(o_col + cc * 32, o);
         tc5::wait_ld();
         if (r < rows) {
 #pragma unroll
@@ -580,7 +569,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_le
   p.num_kv_heads = num_kv_heads;
   p.block_size = block_size;
   p.total_q = total_q;
-  const int rows_per_cta = pa::ptc::BM * (head_dim == 128 ? pa::ptc::Groups<128>::kNWG : pa::ptc::Groups<64>::kNWG);
+  const int rows_per_cta = pa::ptc::BM * pa::ptc::kGroups;
   p.q_tiles = (max_q_len + rows_per_cta - 1) / rows_per_cta;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
