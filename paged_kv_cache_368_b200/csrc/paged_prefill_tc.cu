@@ -218,23 +218,30 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
 #pragma unroll
             for (int q = 0; q < BN / 16; ++q)
               bytes += (bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1)) * (D / 64) * box_bytes;
-            // K first: the score MMA needs only K; V is consumed later.
-            for (int kv = 0; kv < 2; ++kv) {
-              uint64_t* full = kv == 0 ? &k_full[st] : &v_full[st];
-              const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
-              const uint32_t dst = (kv == 0 ? k_s : v_s) + st * L::kKV;
-              mbar_arrive_expect_tx(full, bytes);
+            // K first (the score MMA needs only K): one box per head_dim
+            // half and block, into [half][BN rows][128 B].
+            const uint32_t kdst = k_s + st * L::kKV, vdst = v_s + st * L::kKV;
+            mbar_arrive_expect_tx(&k_full[st], bytes);
 #pragma unroll
-              for (int q = 0; q < BN / 16; ++q) {
-                const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
-                for (int b = 0; b < nb; ++b) {
-                  const int phys = b == 0 ? bb0[q] : bb1[q];
+            for (int q = 0; q < BN / 16; ++q) {
+              const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
+              for (int b = 0; b < nb; ++b) {
+                const int phys = b == 0 ? bb0[q] : bb1[q];
 #pragma unroll
-                  for (int cq = 0; cq < D / 64; ++cq)
-                    tc5::tma_load_4d(dst + cq * (BN * 128) + q * 2048 + b * 1024, map, full, 64 * cq, rr0[q], kvh,
-                                     phys);
-                }
+                for (int cq = 0; cq < D / 64; ++cq)
+                  tc5::tma_load_4d(kdst + cq * (BN * 128) + q * 2048 + b * 1024, &kmap, &k_full[st], 64 * cq, rr0[q],
+                                   kvh, phys);
               }
+            }
+            // V: one box per block covering both head_dim halves, chunk-major
+            // ([16-key chunk][block][half][rows][128 B]).
+            mbar_arrive_expect_tx(&v_full[st], bytes);
+#pragma unroll
+            for (int q = 0; q < BN / 16; ++q) {
+              const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
+              for (int b = 0; b < nb; ++b)
+                tc5::tma_load_5d(vdst + q * (32 * D) + b * (D / 64) * box_bytes, &vmap, &v_full[st], 0, rr0[q], 0, kvh,
+                                 b == 0 ? bb0[q] : bb1[q]);
             }
           }
         }
@@ -282,6 +289,12 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       __syncwarp();
       return true;
     };
+    // V tile, chunk-major: the head_dim halves of a chunk are box_rows * 128 B
+    // apart (LBO) and its two 8-key row groups 1 KB apart, or one block's box
+    // apart when a chunk spans two 8-row blocks (SBO).
+    const int box_rows = p.block_size < 16 ? p.block_size : 16;
+    const uint32_t v_lbo = box_rows * 128;
+    const uint32_t v_sbo = p.block_size >= 16 ? 1024u : uint32_t(D / 64) * 1024u;
     auto issue_pv = [&](int g, int j) -> bool {  // O_g += P(g, j) V_j, P from tensor memory
       const int st = j % STAGES;
       if (!wait_all(&v_full[st], (j / STAGES) & 1)) return false;
@@ -292,7 +305,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       const uint32_t od = tmem + g * L::kColsPerGroup + 2 * BN;
 #pragma unroll
       for (int ks = 0; ks < BN / 16; ++ks) {
-        const uint64_t db = tc5::sw128_desc(vt + ks * (16 * 128), BN * 128, 1024);
+        const uint64_t db = tc5::sw128_desc(vt + ks * (32 * D), v_lbo, v_sbo);
         tc5::mma_ts_if(leader, od, pa + ks * 8, db, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
       }
       tc5::commit_if(leader, pv_done(g, j & 1));
@@ -418,9 +431,13 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
         const int vfirst = max(0, kend - key0);
         const uint32_t vt = v_s + (j % STAGES) * L::kKV;
         const int nvec = (BN - vfirst) * (D / 8);
+        const int box_rows = p.block_size < 16 ? p.block_size : 16;
         for (int i = r; i < nvec; i += BM) {
           const int vr = vfirst + i / (D / 8), c16 = i % (D / 8);
-          sts128(vt + (c16 >> 3) * (BN * 128) + vr * 128 + (((c16 & 7) ^ (vr & 7)) << 4), make_uint4(0, 0, 0, 0));
+          const int kk = vr & 15, vb = kk / box_rows, rr = kk % box_rows;
+          sts128(vt + (vr >> 4) * (32 * D) + (vb * (D / 64) + (c16 >> 3)) * box_rows * 128 + rr * 128 +
+                     (((c16 & 7) ^ (rr & 7)) << 4),
+                 make_uint4(0, 0, 0, 0));
         }
         fence_proxy_async_smem();
       }
@@ -496,6 +513,25 @@ bool make_q_map(CUtensorMap* map, const void* q, int total_q, int heads, int d) 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// V pool [NB][KVH][BS][D] as a 5-D tensor {64 dims, rows, D/64 halves, kv
+// head, block} so that one box brings a block's rows for every head_dim half
+// ([half][rows][128 B], 128-byte swizzle).
+bool make_v_map(CUtensorMap* map, const void* v, int64_t nb, int kvh, int bs, int d) {
+  void* fn_ptr = nullptr;
+  cudaDriverEntryPointQueryResult qr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn_ptr, cudaEnableDefault, &qr) != cudaSuccess ||
+      qr != cudaDriverEntryPointSuccess)
+    return false;
+  auto fn = reinterpret_cast<EncodeTiledFn>(fn_ptr);
+  const cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)(d / 64), (cuuint64_t)kvh, (cuuint64_t)nb};
+  const cuuint64_t strides[4] = {(cuuint64_t)d * 2, 128, (cuuint64_t)bs * d * 2, (cuuint64_t)kvh * bs * d * 2};
+  const cuuint32_t box[5] = {64, (cuuint32_t)(bs < 16 ? bs : 16), (cuuint32_t)(d / 64), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 5, const_cast<void*>(v), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int D>
 pa_status launch_tc(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm, const pa::ptc::Params& p,
                     int dev, cudaStream_t stream) {
@@ -552,7 +588,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const int32_t* cu_q_le
   if (ce != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaGetDevice", ce);
   CUtensorMap km, vm, qm;
   if (!pa::make_cache_map(&km, k_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
-      !pa::make_cache_map(&vm, v_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
+      !make_v_map(&vm, v_cache, num_blocks, num_kv_heads, block_size, head_dim) ||
       !make_q_map(&qm, q, total_q, num_heads, head_dim))
     return pa::fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled rejected a layout", cudaSuccess);
   pa::ptc::Params p;
