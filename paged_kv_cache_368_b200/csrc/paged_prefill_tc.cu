@@ -68,7 +68,7 @@ struct Lay {
   // p_full[2], pv_done[2]; mma_done
   static constexpr int kBars = 1 + 3 * STAGES + NWG * 6 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kBars * 8 + 16;
-  static constexpr int kThreads = (4 + 4 * NWG) * 32;  // warps 0-3: TMA, MMA, idle, idle
+  static constexpr int kThreads = (4 + 4 * NWG) * 32;  // warps 0-3: TMA (Q, K), MMA, TMA (V), idle
   // Tensor memory per group: S0 | S1 | O.  P of tile j (16-bit, two per
   // column) overwrites the front of S(j & 1) once the softmax has read it.
   static constexpr uint32_t kColsPerGroup = 2 * BN + D;
@@ -161,12 +161,16 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
   const bool active = ntiles > 0;
   const uint32_t q_s = base, k_s = base + L::kOffK, v_s = base + L::kOffV;
 
-  if (active && warp == 0) {
-    // ------------------------------------------------------------- producer
+  if (active && (warp == 0 || warp == 2)) {
+    // ------------------------------------------------------------- producers
+    // Warp 0 copies Q and every K tile, warp 2 every V tile: one thread
+    // issues a TMA box only every 100-200 cycles, so the two streams go out
+    // in parallel.  Both walk the same block-table entries.
+    const bool kprod = warp == 0;
     const int bs = p.block_size;
     const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
     const uint32_t box_bytes = (bs < 16 ? bs : 16) * 128;
-    if (lane == 0) {
+    if (kprod && lane == 0) {
       uint32_t qbytes = 0;
       for (int g = 0; g < NWG; ++g)
         if (g_rows(g) > 0) qbytes += L::kQ;
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
           if (t0 + 8 < kend) b1 = __ldg(row + 2 * c + 1);
         }
         if (!(b0 >= 0 && b0 < p.num_blocks && (b1 == -1 || (b1 >= 0 && b1 < p.num_blocks)))) {
-          set_err(p.err_flags, PA_ERRF_BLOCK_RANGE);
+          if (kprod) set_err(p.err_flags, PA_ERRF_BLOCK_RANGE);
           b0 = b1 = -1;
         }
       }
@@ -218,30 +222,33 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
 #pragma unroll
             for (int q = 0; q < BN / 16; ++q)
               bytes += (bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1)) * (D / 64) * box_bytes;
-            // K first (the score MMA needs only K): one box per head_dim
-            // half and block, into [half][BN rows][128 B].
-            const uint32_t kdst = k_s + st * L::kKV, vdst = v_s + st * L::kKV;
-            mbar_arrive_expect_tx(&k_full[st], bytes);
+            if (kprod) {
+              // K: one box per head_dim half and block, into [half][BN rows][128 B].
+              const uint32_t kdst = k_s + st * L::kKV;
+              mbar_arrive_expect_tx(&k_full[st], bytes);
 #pragma unroll
-            for (int q = 0; q < BN / 16; ++q) {
-              const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
-              for (int b = 0; b < nb; ++b) {
-                const int phys = b == 0 ? bb0[q] : bb1[q];
+              for (int q = 0; q < BN / 16; ++q) {
+                const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
+                for (int b = 0; b < nb; ++b) {
+                  const int phys = b == 0 ? bb0[q] : bb1[q];
 #pragma unroll
-                for (int cq = 0; cq < D / 64; ++cq)
-                  tc5::tma_load_4d(kdst + cq * (BN * 128) + q * 2048 + b * 1024, &kmap, &k_full[st], 64 * cq, rr0[q],
-                                   kvh, phys);
+                  for (int cq = 0; cq < D / 64; ++cq)
+                    tc5::tma_load_4d(kdst + cq * (BN * 128) + q * 2048 + b * 1024, &kmap, &k_full[st], 64 * cq,
+                                     rr0[q], kvh, phys);
+                }
               }
-            }
-            // V: one box per block covering both head_dim halves, chunk-major
-            // ([16-key chunk][block][half][rows][128 B]).
-            mbar_arrive_expect_tx(&v_full[st], bytes);
+            } else {
+              // V: one box per block covering both head_dim halves, chunk-major
+              // ([16-key chunk][block][half][rows][128 B]).
+              const uint32_t vdst = v_s + st * L::kKV;
+              mbar_arrive_expect_tx(&v_full[st], bytes);
 #pragma unroll
-            for (int q = 0; q < BN / 16; ++q) {
-              const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
-              for (int b = 0; b < nb; ++b)
-                tc5::tma_load_5d(vdst + q * (32 * D) + b * (D / 64) * box_bytes, &vmap, &v_full[st], 0, rr0[q], 0, kvh,
-                                 b == 0 ? bb0[q] : bb1[q]);
+              for (int q = 0; q < BN / 16; ++q) {
+                const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
+                for (int b = 0; b < nb; ++b)
+                  tc5::tma_load_5d(vdst + q * (32 * D) + b * (D / 64) * box_bytes, &vmap, &v_full[st], 0, rr0[q], 0,
+                                   kvh, b == 0 ? bb0[q] : bb1[q]);
+              }
             }
           }
         }
@@ -254,10 +261,8 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     // The last tiles' copies have landed (always, on the normal path) before
     // the CTA may exit.
     if (lane == 0) {
-      for (int j = max(0, ntiles - STAGES); j < ntiles; ++j) {
-        tc5::wait(&k_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
-        tc5::wait(&v_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
-      }
+      for (int j = max(0, ntiles - STAGES); j < ntiles; ++j)
+        tc5::wait(kprod ? &k_full[j % STAGES] : &v_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
     }
   } else if (active && warp == 1) {
     // ------------------------------------------------------------- MMA issue
