@@ -5,22 +5,28 @@
 // head_dim] call; each row the section 1.1 formula of "【infra之路】10-
 // PagedAttention 与 KV Cache 管理", restricted to positions up to its own).
 //
-// One CTA per (128-row query tile, q-head, sequence), 8 warps:
-//   warp 0      TMA producer: the Q tile once (3-D map over [token][head][d]),
-//               then K and V of 64-key tiles, 16 rows per box read through
-//               the block table, into a 3-stage ring;
-//   warp 1      allocates tensor memory and issues the MMAs (one thread):
-//               S_j = Q K_j^T (M 128, N 64) into one of two TMEM buffers, and
-//               O += P_j V_j (M 128, N head_dim) into a TMEM accumulator;
-//               S_{j+1} is issued before waiting for P_j, so it overlaps the
-//               softmax of tile j;
-//   warps 4-7   softmax: thread t owns query row t (TMEM lane t).  It reads
-//               S_j, applies the causal mask, keeps a running max that is
-//               only moved when it grows by more than 2^8 (so the O rescale in
-//               tensor memory is rare), writes P_j (bf16/fp16) into a swizzled
-//               shared tile, and at the end reads O and divides by the sum.
-// All operand tiles are 128-byte-swizzled, the layout TMA writes and the MMA
-// descriptors name directly.
+// One CTA per (256 query rows, q-head, sequence), 12 warps:
+//   warp 0      TMA: both 128-row Q tiles once (3-D map over [token][head][d]),
+//               then the K tiles of 64 keys, one 16-row box per block and
+//               head_dim half, read through the block table;
+//   warp 2      TMA: the V tiles, one 5-D box per block covering both
+//               head_dim halves (chunk-major layout);
+//               K and V go into a ring 5 tiles deep (8 at head_dim 64);
+//   warp 1      allocates tensor memory and runs the MMA schedule as a whole
+//               warp, one elected lane issuing: S = Q K^T (M 128, N 64, both
+//               operands in shared memory) into one of two TMEM buffers per
+//               query tile, and O += P V (M 128, N head_dim) with P read from
+//               tensor memory; per query tile, P.V of tile j comes before the
+//               scores of tile j+2, which reuse P's columns;
+//   warps 4-7,  softmax of query tiles 0 and 1: thread t owns query row t
+//   8-11        (TMEM lane t).  It reads S_j, masks on tiles that reach its
+//               first row, keeps a reference max that moves only when it grows
+//               by more than 2^8 (so the O rescale in tensor memory is rare),
+//               writes P_j as 16-bit pairs over S_j, and at the end reads O and
+//               divides by the row sum;
+//   warp 3      idle.
+// Shared-memory operand tiles are 128-byte-swizzled, the layout TMA writes
+// and the MMA descriptors name directly.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -60,7 +66,8 @@ struct Lay {
   static constexpr int NWG = kGroups;
   static constexpr int STAGES = D == 128 ? 5 : 8;  // K/V ring depth (tiles in flight)
   static constexpr int kQ = BM * D * 2;   // per group: [D/64][BM rows][128 B]
-  static constexpr int kKV = BN * D * 2;  // one K or V tile: [D/64][BN rows][128 B]
+  // one K or V tile; K: [D/64][BN rows][128 B], V: [BN/16 chunks][block][D/64][rows][128 B]
+  static constexpr int kKV = BN * D * 2;
   static constexpr int kOffK = NWG * kQ;
   static constexpr int kOffV = kOffK + STAGES * kKV;
   static constexpr int kOffBar = kOffV + STAGES * kKV;
