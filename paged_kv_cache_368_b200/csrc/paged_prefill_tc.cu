@@ -71,9 +71,9 @@ struct Lay {
   static constexpr int kOffK = NWG * kQ;
   static constexpr int kOffV = kOffK + STAGES * kKV;
   static constexpr int kOffBar = kOffV + STAGES * kKV;
-  // barriers: q_full, k_full[S], v_full[S], kv_empty[S]; per group s_full[2],
-  // p_full[2], pv_done[2]; mma_done
-  static constexpr int kBars = 1 + 3 * STAGES + NWG * 6 + 1;
+  // barriers: q_full, kv_full[S] (one arrival per producer warp), kv_empty[S];
+  // per group s_full[2], p_full[2], pv_done[2]; mma_done
+  static constexpr int kBars = 1 + 2 * STAGES + NWG * 6 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kBars * 8 + 16;
   static constexpr int kThreads = (4 + 4 * NWG) * 32;  // warps 0-3: TMA (Q, K), MMA, TMA (V), idle
   // Tensor memory per group: S0 | S1 | O.  P of tile j (16-bit, two per
@@ -97,9 +97,8 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
   uint8_t* smem = smem_raw + (base - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + STAGES;
-  uint64_t* kv_empty = v_full + STAGES;
+  uint64_t* kv_full = bars + 1;  // K and V of a tile: the score MMA waits for both
+  uint64_t* kv_empty = kv_full + STAGES;
   // Group g owns bars [6g, 6g+6); double-buffered barriers are indexed by the
   // tile's parity, so no waiter can fall two phases behind.
   uint64_t* grp_bars = kv_empty + STAGES;
@@ -120,8 +119,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     prefetch_tensormap(&qmap);
     mbar_init(q_full, 1);
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_full[i], 2);
       mbar_init(&kv_empty[i], 1);
     }
     for (int g = 0; g < NWG; ++g) {
@@ -232,7 +230,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
             if (kprod) {
               // K: one box per head_dim half and block, into [half][BN rows][128 B].
               const uint32_t kdst = k_s + st * L::kKV;
-              mbar_arrive_expect_tx(&k_full[st], bytes);
+              mbar_arrive_expect_tx(&kv_full[st], bytes);
 #pragma unroll
               for (int q = 0; q < BN / 16; ++q) {
                 const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
@@ -240,7 +238,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
                   const int phys = b == 0 ? bb0[q] : bb1[q];
 #pragma unroll
                   for (int cq = 0; cq < D / 64; ++cq)
-                    tc5::tma_load_4d(kdst + cq * (BN * 128) + q * 2048 + b * 1024, &kmap, &k_full[st], 64 * cq,
+                    tc5::tma_load_4d(kdst + cq * (BN * 128) + q * 2048 + b * 1024, &kmap, &kv_full[st], 64 * cq,
                                      rr0[q], kvh, phys);
                 }
               }
@@ -248,12 +246,12 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
               // V: one box per block covering both head_dim halves, chunk-major
               // ([16-key chunk][block][half][rows][128 B]).
               const uint32_t vdst = v_s + st * L::kKV;
-              mbar_arrive_expect_tx(&v_full[st], bytes);
+              mbar_arrive_expect_tx(&kv_full[st], bytes);
 #pragma unroll
               for (int q = 0; q < BN / 16; ++q) {
                 const int nb = bb0[q] < 0 ? 0 : (bb1[q] >= 0 ? 2 : 1);
                 for (int b = 0; b < nb; ++b)
-                  tc5::tma_load_5d(vdst + q * (32 * D) + b * (D / 64) * box_bytes, &vmap, &v_full[st], 0, rr0[q], 0,
+                  tc5::tma_load_5d(vdst + q * (32 * D) + b * (D / 64) * box_bytes, &vmap, &kv_full[st], 0, rr0[q], 0,
                                    kvh, b == 0 ? bb0[q] : bb1[q]);
               }
             }
@@ -269,7 +267,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     // the CTA may exit.
     if (lane == 0) {
       for (int j = max(0, ntiles - STAGES); j < ntiles; ++j)
-        tc5::wait(kprod ? &k_full[j % STAGES] : &v_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+        tc5::wait(&kv_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
     }
   } else if (active && warp == 1) {
     // ------------------------------------------------------------- MMA issue
@@ -287,7 +285,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     };
     auto issue_qk = [&](int g, int j) -> bool {  // S(g, j&1) = Q_g K_j^T
       const int st = j % STAGES;
-      if (!wait_all(&k_full[st], (j / STAGES) & 1)) return false;
+      if (!wait_all(&kv_full[st], (j / STAGES) & 1)) return false;
       tc5::fence_after();
       const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
       const uint32_t sd = tmem + g * L::kColsPerGroup + (j & 1) * BN;
@@ -309,7 +307,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     const uint32_t v_sbo = p.block_size >= 16 ? 1024u : uint32_t(D / 64) * 1024u;
     auto issue_pv = [&](int g, int j) -> bool {  // O_g += P(g, j) V_j, P from tensor memory
       const int st = j % STAGES;
-      if (!wait_all(&v_full[st], (j / STAGES) & 1)) return false;
+      // V landed with K: the scores of tile j, issued earlier, waited for both.
       if (!wait_all(p_full(g, j & 1), (j >> 1) & 1)) return false;
       tc5::fence_after();
       const uint32_t vt = v_s + st * L::kKV;
@@ -435,7 +433,7 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       // in the CTA's last tile (once its copy has landed), and its P.V is
       // issued before the others'.
       if (g == lastg && key0 + BN > kend) {
-        const bool vin = tc5::wait(&v_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+        const bool vin = tc5::wait(&kv_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
         if (!__all_sync(kFull, vin)) {
           ok = false;
           break;
