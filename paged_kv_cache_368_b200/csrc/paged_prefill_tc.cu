@@ -283,9 +283,15 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       const bool got = tc5::wait(bar, parity, kWaitNs);
       return __all_sync(kFull, got);
     };
+    int kv_seen = -1;  // highest tile whose copies this warp has already waited for
     auto issue_qk = [&](int g, int j) -> bool {  // S(g, j&1) = Q_g K_j^T
       const int st = j % STAGES;
-      if (!wait_all(&kv_full[st], (j / STAGES) & 1)) return false;
+      // Tiles are waited for in increasing order; the second group's scores
+      // of the same tile skip the (already satisfied) wait.
+      if (j > kv_seen) {
+        if (!wait_all(&kv_full[st], (j / STAGES) & 1)) return false;
+        kv_seen = j;
+      }
       tc5::fence_after();
       const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
       const uint32_t sd = tmem + g * L::kColsPerGroup + (j & 1) * BN;
