@@ -297,6 +297,19 @@ PA_API pa_status pa_bm_prepare_decode(pa_block_manager* m, const int64_t* seq_id
 PA_API pa_status pa_bm_swap_sequence(pa_block_manager* from, pa_block_manager* to, int64_t seq_id, int64_t* pairs,
                               int64_t max_pairs, int64_t* num_pairs);
 
+/*
+ * pa_selftest_wait_timeout -- checks, on the device, the bounded barrier wait
+ * that every kernel above relies on (the pages have no counterpart).  One
+ * CTA waits on two shared-memory barriers that nothing ever completes, one
+ * with each wait flavour the kernels use (plain probe loop; suspending
+ * probe), each limited to `limit_ns` nanoseconds (1 .. 1e8).  Each wait must
+ * give up, after which PA_ERRF_TIMEOUT is OR-ed into err_flags[0] (plain)
+ * and err_flags[1] (suspending), int32 device words owned by the caller, and
+ * the kernel returns: no trap, the context stays usable.  Asynchronous on
+ * `stream`; PA_ERR_INVALID for a NULL err_flags or a limit out of range.
+ */
+PA_API pa_status pa_selftest_wait_timeout(uint64_t limit_ns, int32_t* err_flags, pa_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 PA_API const char* pa_status_string(pa_status status);
 

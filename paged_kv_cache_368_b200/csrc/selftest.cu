@@ -1,0 +1,38 @@
+// Self-test of the bounded barrier wait every kernel of the library relies on
+// (no counterpart on the pages): one CTA waits on shared-memory barriers that
+// nothing ever completes and must give up after the given limit, flag the
+// timeout and return, leaving the context usable.
+#include "pa_host.h"
+#include "tcgen05.cuh"
+
+namespace pa {
+namespace {
+
+__global__ void __launch_bounds__(32, 1) wait_timeout_kernel(uint64_t limit_ns, int32_t* err_flags) {
+  __shared__ __align__(8) uint64_t bars[2];
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  // Phase 0 of either barrier never completes: no thread arrives on it.  Both
+  // wait flavours used by the kernels are exercised: the plain probe loop
+  // (decode) and the suspending probe (tensor-core prefill).
+  const bool plain = mbar_wait_bounded(&bars[0], 0, limit_ns);
+  const bool suspending = tc5::wait(&bars[1], 0, limit_ns);
+  if (threadIdx.x == 0) {
+    if (!plain) set_err(err_flags, PA_ERRF_TIMEOUT);
+    if (!suspending) set_err(err_flags + 1, PA_ERRF_TIMEOUT);
+  }
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" pa_status pa_selftest_wait_timeout(uint64_t limit_ns, int32_t* err_flags, pa_stream_t stream) {
+  if (!err_flags || limit_ns == 0 || limit_ns > 100000000ull) return PA_ERR_INVALID;
+  pa::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, err_flags);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : pa::fail(PA_ERR_CUDA, "launching wait_timeout_kernel", e);
+}

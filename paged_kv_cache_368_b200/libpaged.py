@@ -28,7 +28,8 @@ SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_
            "pa_decode_step_host", "pa_step_inputs_layout", "pa_prefill", "pa_prefill_mma", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
            "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slot",
            "pa_bm_free_sequence", "pa_bm_context_len", "pa_bm_block_table", "pa_bm_blocks_needed_to_append",
-           "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_status_string", "pa_version", "pa_last_error")
+           "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_selftest_wait_timeout", "pa_status_string",
+           "pa_version", "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -74,6 +75,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, f).argtypes = [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32,
                                     _i32, _i32, _i64, _i32, _vp, _vp]
         getattr(lib, f).restype = _i32
+    lib.pa_selftest_wait_timeout.argtypes = [_c.c_uint64, _vp, _vp]
+    lib.pa_selftest_wait_timeout.restype = _i32
     lib.pa_status_string.argtypes = [_i32]
     lib.pa_status_string.restype = _c.c_char_p
     lib.pa_version.argtypes = []
@@ -300,6 +303,16 @@ def _setup_block_api(lib):
         getattr(lib, f).restype = _i32
     lib._block_api = True
     return lib
+
+
+def selftest_wait_timeout(err_flags: torch.Tensor, limit_ns: int = 2_000_000, stream=None) -> None:
+    """Run the bounded-wait self-test: ``err_flags`` (int32, 2 words, on the
+    device) receives ``ERRF_TIMEOUT`` in each word once its wait has given up."""
+    if err_flags.dtype != torch.int32 or err_flags.numel() < 2:
+        raise ValueError("err_flags must be an int32 device tensor of at least 2 words")
+    st = load().pa_selftest_wait_timeout(int(limit_ns), _dev_ptr(err_flags, "err_flags"), _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_selftest_wait_timeout")
 
 
 def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_pairs: torch.Tensor,

@@ -121,6 +121,13 @@ def test_prefill_host_checks(lib, entry):
         assert call(scale=-0.1) == U
 
 
+def test_selftest_host_checks(lib):
+    I = libpaged.PA_ERR_INVALID
+    assert lib.pa_selftest_wait_timeout(1000, None, None) == I  # no flag words
+    assert lib.pa_selftest_wait_timeout(0, 16, None) == I  # zero limit
+    assert lib.pa_selftest_wait_timeout(200_000_000, 16, None) == I  # above 0.1 s
+
+
 def test_workspace_size_rejects_bad_shapes(lib):
     assert lib.pa_decode_workspace_size(4, 6, 4, 128, 100) == 0
     assert lib.pa_decode_workspace_size(4, 32, 2, 128, 100) == 0  # group of 16
