@@ -73,3 +73,53 @@ def test_empty_rows_and_sequences():
     wl, k, v, cu, q = _case(9, 3, 2, 2, 8, 4, [6, 7, 3], [0, 2, 0])
     out = opa.prefill(q, cu, k, v, wl.block_tables, wl.context_lens, wl.scale, "f16")
     assert out.shape == (2, 2, 8) and np.isfinite(out).all()
+
+
+# ------------------------------------------------------------------ planted mistakes
+# Each mutant is a plausible slip in the prefill oracle (planted here, on the
+# CPU); at least one of the pins above must reject it.
+
+def _mutant(last_offset=1, ignore_prefix=False, no_causal=False):
+    def prefill(q, cu_q, k_cache, v_cache, block_tables, context_lens, scale, dtype):
+        total, H, d = q.shape
+        out = np.zeros((total, H, d))
+        sc = float(np.float32(scale))
+        for s in range(len(context_lens)):
+            lo, hi, L = int(cu_q[s]), int(cu_q[s + 1]), int(context_lens[s])
+            n = hi - lo
+            if n == 0 or L == 0:
+                continue
+            k64 = opa.gather(k_cache, block_tables[s], L, dtype)
+            v64 = opa.gather(v_cache, block_tables[s], L, dtype)
+            for i in range(n):
+                p = i if ignore_prefix else L - n + i
+                end = L if no_causal else min(L, max(1, p + last_offset))
+                out[lo + i] = opa.attend(opa.widen(q[lo + i], dtype), k64[:, :end], v64[:, :end], sc)
+        return out
+    return prefill
+
+
+PREFILL_MUTANTS = {
+    "excludes own position": _mutant(last_offset=0),
+    "sees the next position": _mutant(last_offset=2),
+    "ignores the cached prefix": _mutant(ignore_prefix=True),
+    "no causal mask": _mutant(no_causal=True),
+}
+PREFILL_PINS = (test_single_token_rows_equal_decode, test_full_prompt_equals_causal_sdpa, test_brute_force_tiny_chunk)
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for pin in PREFILL_PINS:
+        pin()
+
+
+@pytest.mark.parametrize("name", sorted(PREFILL_MUTANTS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    monkeypatch.setattr(opa, "prefill", PREFILL_MUTANTS[name])
+    caught = 0
+    for pin in PREFILL_PINS:
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"mutant '{name}' passed every prefill pin"
