@@ -508,9 +508,65 @@ def run_block_ops(args):
                                     "contiguous_memcpy_gbs": sw / (ms_d2h * 1e-3) / 1e9},
         "swap_in_from_pinned_host": {"us_per_call": ms_in * 1e3, "bytes": sw, "gbs": sw / (ms_in * 1e-3) / 1e9,
                                      "contiguous_memcpy_gbs": sw / (ms_h2d * 1e-3) / 1e9},
+        "roofline": {"bound": "hbm", "achieved": copy_gbs, "peak": peak, "unit": "GB/s", "frac": copy_gbs / peak,
+                     "traffic": None, "kernel": "pa_copy_blocks (read + write bytes)"},
     }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = block_copy_cpu_baseline(kvh, bs, d)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def block_copy_cpu_baseline(kvh, bs, d, budget_s=4.0):
+    """The oracle's copy_blocks (NumPy, as it stands: it copies the pool it is
+    given, then the pairs) on a 512-block host pool with 128 pairs, counted like
+    the GPU number (read + write bytes of the copied blocks)."""
+    from oracle.block_manager import copy_blocks
+
+    rng = np.random.default_rng(368)
+    pool = rng.integers(0, 1 << 16, size=(512, kvh, bs, d), dtype=np.uint16)
+    ids = rng.permutation(512)
+    pairs = list(zip(ids[:128].tolist(), ids[128:256].tolist()))
+    t, reps = time_passes(lambda: copy_blocks(pool, pairs), budget_s)
+    nbytes = 2 * 128 * kvh * bs * d * 2
+    return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"oracle copy_blocks on a {pool.nbytes >> 20} MiB host pool, 128 pairs, median of {reps} passes",
+            "host_cpus": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
+
+
+def prefill_cpu_baseline(wl, q, qlen, ctx, H, KVH, D, dtype, budget_s=4.0):
+    """The float64 oracle on a bounded sample of a prefill workload: the first
+    new rows of sequence 0 for the q-heads of kv-head 0, sized to a few
+    seconds of host time."""
+    import torch
+
+    import oracle
+
+    G = H // KVH
+    kp, vp = wl.full_pool(poison=False)
+    kp, vp = np.ascontiguousarray(kp[:, :1]), np.ascontiguousarray(vp[:, :1])
+    n0, c0 = qlen[0], ctx[0]
+
+    def sample(rows):
+        qs = q[:rows, :G].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        cu = np.array([0, rows], dtype=np.int32)
+        cl = np.array([c0 - n0 + rows], dtype=np.int32)
+        pos = np.arange(c0 - n0, c0 - n0 + rows, dtype=np.float64)
+        fl = float(4.0 * D * G * (pos + 1).sum())
+        return (lambda: oracle.prefill(qs, cu, kp, vp, wl.block_tables[:1], cl, wl.scale, dtype)), fl
+
+    rows = 1  # double the sample until one pass takes about a sixth of the budget
+    while True:
+        run, fl = sample(rows)
+        t1, _ = time_passes(run, 0.0)
+        if t1 > budget_s / 6 or rows >= n0:
+            break
+        rows = min(n0, rows * 2)
+    t, reps = time_passes(run, budget_s)
+    return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"float64 NumPy oracle, sequence 0 rows 0..{rows - 1} of {n0}, the {G} q-heads of "
+                       f"kv-head 0, median of {reps} passes"),
+            "host_cpus": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
 
 
 def run_prefill(args):
@@ -582,9 +638,14 @@ def run_prefill(args):
             pos = np.arange(c - n, c, dtype=np.float64)
             flops += float(4.0 * D * H * (pos + 1).sum())
         tf = flops / (ms * 1e-3) / 1e12
-        results.append({"workload": name, "us": ms * 1e3, "tflops": tf, "frac_of_bf16_peak": tf / peak,
-                        "kv_bytes_logical": wl.kv_bytes(), "flops": flops, "kernel": "tcgen05",
-                        "mma_sync_us": ms_mma * 1e3, "mma_sync_tflops": flops / (ms_mma * 1e-3) / 1e12})
+        res = {"workload": name, "us": ms * 1e3, "tflops": tf, "frac_of_bf16_peak": tf / peak,
+               "kv_bytes_logical": wl.kv_bytes(), "flops": flops, "kernel": "tcgen05",
+               "mma_sync_us": ms_mma * 1e3, "mma_sync_tflops": flops / (ms_mma * 1e-3) / 1e12,
+               "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                            "traffic": None, "traffic_note": "kernel changed since the committed ncu capture"}}
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = prefill_cpu_baseline(wl, q, qlen, ctx, H, KVH, D, dtype)
+        results.append(res)
     line = {"metric": "pa_prefill causal attention TFLOP/s", "op": "prefill", "n_gpus": 1, "steps": K, "warmup": W,
             "peak_tflops": peak, "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)",
             "results": results}
