@@ -275,8 +275,12 @@ PA_API int64_t pa_bm_context_len(const pa_block_manager* m, int64_t seq_id);
 PA_API pa_status pa_bm_block_table(const pa_block_manager* m, int64_t seq_id, int32_t* table, int max_blocks,
                             int* num_blocks);
 
-/* Free blocks one more token for each listed sequence would take (for
- * admission control, the tutorial's section 6 scheduler); -1 on bad ids. */
+/* Free blocks that appending one more token to each listed sequence takes
+ * (admission control, the tutorial's section 6 scheduler): one per sequence
+ * whose last block is full, plus, for a partly filled last block held by r
+ * sequences of which k are listed, min(k, r-1) copies (the last writer keeps
+ * the block).  Exactly what pa_bm_prepare_decode on the same batch takes;
+ * -1 on bad ids. */
 PA_API int64_t pa_bm_blocks_needed_to_append(const pa_block_manager* m, const int64_t* seq_ids, int num_seqs);
 
 /* One decode step for a batch: appends one token to each sequence and writes

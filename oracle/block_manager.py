@@ -1,7 +1,8 @@
 """Reference model of the block manager and of whole-block copies.
 
-TEST INFRASTRUCTURE, NOT PRODUCT CODE: only ``tests/`` may use it.  It shares
-no code with the library's C++ block manager.
+TEST INFRASTRUCTURE, NOT PRODUCT CODE: only ``tests/`` and the CPU-baseline
+timing in ``bench.py`` may use it.  It shares no code with the library's C++
+block manager or its copy kernels.
 
 Follows:
 * "PagedAttention：KV Cache 的分页革命", section Runtime 如何管理 KV Block: a
@@ -12,13 +13,22 @@ Follows:
   block table grows by one physical block when its last block is full),
   section 4.3 (requests sharing a prefix, and beams, point at the same
   physical blocks; a shared block is copied before it is written; preempted
-  requests are swapped to CPU memory and back).
+  requests are swapped to CPU memory and back), section 6 (the scheduler
+  admits work by the number of free blocks).
 
 Policies the pages leave open, read the plainest way: the free block with the
 smallest id is taken first; running out of blocks is an error that changes
-nothing.
+nothing; a sequence moved to another pool gets a fresh block there for each
+of its blocks, so blocks it shared stay with the other holders and are not
+shared in the new pool.
+
+Pinned in ``tests/test_oracle_block_pins.py`` against hand-worked scenarios
+(``tests/golden/block_manager_*.json``, ``tests/golden/block_copy_example.json``)
+with planted mistakes that the pins must reject.
 """
 from __future__ import annotations
+
+import copy
 
 import numpy as np
 
@@ -85,11 +95,18 @@ class BlockManagerModel:
         del self.lens[seq]
 
     def blocks_needed_to_append(self, seqs):
-        n = 0
+        """Free blocks that appending one token to each of `seqs` takes (the
+        admission count of the tutorial's section 6 scheduler).  Defined by
+        doing it: the appends run on a copy whose pool can never run out, and
+        the blocks they took are counted.  So a shared last block costs one
+        copy per sharer in the batch except the one left holding it alone."""
+        sim = copy.deepcopy(self)
+        sim.num_blocks += len(seqs)
+        sim.refs += [0] * len(seqs)
+        before = len(sim.free_blocks())
         for s in seqs:
-            if self.lens[s] % self.block_size == 0 or self.refs[self.tables[s][-1]] > 1:
-                n += 1
-        return n
+            sim.append_slot(s)
+        return before - len(sim.free_blocks())
 
     def swap_to(self, other: "BlockManagerModel", seq):
         """Move `seq` into `other`'s pool; returns [(block here, block there)]."""

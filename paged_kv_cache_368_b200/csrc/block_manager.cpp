@@ -165,12 +165,26 @@ extern "C" pa_status pa_bm_block_table(const pa_block_manager* m, int64_t seq_id
 
 extern "C" int64_t pa_bm_blocks_needed_to_append(const pa_block_manager* m, const int64_t* seq_ids, int num_seqs) {
   if (!m || (num_seqs > 0 && !seq_ids)) return -1;
+  // A full last block (or none) takes a new block.  A partly filled last
+  // block held by r sequences is copied by each holder that writes while
+  // others still hold it: k holders appending in one batch take min(k, r-1)
+  // blocks, the last writer keeps the original.
   int64_t need = 0;
+  std::unordered_map<int64_t, int32_t> copies;  // shared last block -> copies taken so far
   for (int i = 0; i < num_seqs; ++i) {
     auto it = m->seqs.find(seq_ids[i]);
     if (it == m->seqs.end()) return -1;
     const auto& s = it->second;
-    if (s.len % m->block_size == 0 || m->refcount[s.blocks.back()] > 1) ++need;
+    if (s.len % m->block_size == 0) {
+      ++need;
+      continue;
+    }
+    const int64_t last = s.blocks.back();
+    int32_t& taken = copies[last];
+    if (m->refcount[last] - taken > 1) {
+      ++taken;
+      ++need;
+    }
   }
   return need;
 }

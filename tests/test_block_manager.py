@@ -1,13 +1,13 @@
 """The C++ block manager (through the C ABI, no GPU needed) against the
 pages' lifecycle: a hand-worked scenario, a reference model on random
 operation sequences, and invariants."""
-import json
-import os
 import random
 
 import numpy as np
 import pytest
 
+from block_scenarios import LibraryAdapter, ModelAdapter, golden, run_lifecycle_scenario, run_swap_scenario
+from oracle import block_manager as obm
 from oracle.block_manager import BlockManagerModel, OutOfBlocks
 from paged_kv_cache_368_b200 import build as pbuild
 from paged_kv_cache_368_b200 import libpaged
@@ -19,45 +19,35 @@ def _lib():
     libpaged.load()
 
 
-def _golden():
-    with open(os.path.join(os.path.dirname(__file__), "golden", "block_manager_scenario.json")) as f:
-        return json.load(f)
-
-
-def _run_scenario(mgr, g, is_model):
-    for st in g["steps"]:
-        if st["op"] == "add":
-            mgr.add(st["seq"], st["tokens"])
-        elif st["op"] == "fork":
-            mgr.fork(st["parent"], st["child"])
-        elif st["op"] == "append":
-            if is_model:
-                slot, cow = mgr.append_slot(st["seq"])
-            else:
-                slot, src, dst = mgr.append_slot(st["seq"])
-                cow = (src, dst) if src >= 0 else None
-            assert slot == st["slot"], st
-            assert (list(cow) if cow else None) == st["cow"], st
-        elif st["op"] == "free":
-            mgr.free(st["seq"])
-            n = len(mgr.free_blocks()) if is_model else mgr.num_free
-            assert n == st["num_free"]
-        if "table" in st:
-            seq = st.get("seq", st.get("child"))
-            t = mgr.tables[seq] if is_model else mgr.block_table(seq)
-            assert t == st["table"], st
-    n = len(mgr.free_blocks()) if is_model else mgr.num_free
-    assert n == g["final_num_free"]
-
-
 def test_worked_scenario_model():
-    g = _golden()
-    _run_scenario(BlockManagerModel(g["num_blocks"], g["block_size"]), g, True)
+    run_lifecycle_scenario(lambda n, bs: ModelAdapter(obm, n, bs), golden("block_manager_scenario.json"))
 
 
 def test_worked_scenario_library():
-    g = _golden()
-    _run_scenario(libpaged.BlockManager(g["num_blocks"], g["block_size"]), g, False)
+    run_lifecycle_scenario(LibraryAdapter, golden("block_manager_scenario.json"))
+
+
+def test_swap_and_admission_scenario_library():
+    """The hand-worked two-pool scenario (admission counts, swapping out and
+    back, no sharing after the round trip) on the C++ manager."""
+    run_swap_scenario(LibraryAdapter, golden("block_manager_swap_scenario.json"))
+
+
+def test_prepare_decode_admits_exactly_what_it_takes():
+    """Two sharers of one partly filled block and a sequence with a full
+    block need two free blocks, not three: with exactly two free the batch is
+    admitted and leaves none."""
+    lib = libpaged.BlockManager(6, 4)
+    lib.add(0, 6)    # blocks 0, 1 (block 1 partly filled)
+    lib.fork(0, 1)   # shares 0, 1
+    lib.add(2, 8)    # blocks 2, 3 (full)
+    assert lib.num_free == 2
+    assert lib.blocks_needed_to_append([0, 1, 2]) == 2
+    tables, ctx, slots, cow = lib.prepare_decode([0, 1, 2], 4)
+    assert lib.num_free == 0
+    assert cow.tolist() == [[1, 4]]          # sequence 0 copies block 1 into block 4
+    assert slots.tolist() == [4 * 4 + 2, 1 * 4 + 2, 5 * 4 + 0]
+    assert ctx.tolist() == [7, 7, 9]
 
 
 def _check_invariants(model: BlockManagerModel):
