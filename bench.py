@@ -2,8 +2,8 @@
 """Benchmark of one PagedAttention decode step on B200.
 
 A step is the whole hot path over one batch: the cache append
-(pa_reshape_and_cache) followed by paged decode attention (pa_decode: the
-split-context kernel plus its log-sum-exp merge).  Default workload: the
+(pa_reshape_and_cache) followed by paged decode attention (pa_decode: one
+split-context kernel launch whose log-sum-exp merge runs inside it).  Default workload: the
 LLaMA-7B-shaped layer (32 sequences, 32 q / 32 kv heads, head_dim 128,
 block_size 16, context lengths uniform in [128, 2048], fp16, a shuffled pool
 of 8400 blocks).
@@ -16,6 +16,10 @@ Metric: effective HBM bandwidth = logical K+V bytes the step reads
 Multi-GPU (torchrun, one process per GPU): every rank runs an independent
 replica of the workload (decode shards over sequences with no exchange);
 `value` is the bytes of all ranks / the slowest rank's time.
+
+On one GPU the line also carries `per_config`: the same timings for the other
+workloads (the GQA LLaMA-3-8B layer, the LLaMA-13B layer at block sizes 8, 16,
+32 and 64, the long-context shared-prefix layer and the tiny case).
 """
 from __future__ import annotations
 
@@ -43,8 +47,8 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 
 # DRAM traffic of one decode-kernel launch (dram__bytes_read.sum +
-# dram__bytes_write.sum, ncu --set full, profiles/paged_decode_*.md), keyed by
-# workload; reported only while the decode kernel's device sources hash to `src`.
+# dram__bytes_write.sum from one ncu --set full capture), keyed by workload;
+# reported only while the decode kernel's device sources hash to `src`.
 NCU_TRAFFIC = {
     "llama7b-mha": {"bytes": 584_963_840 + 4_026_112, "src": "f65eb04587b47385"},
     "llama3-8b-gqa": {"bytes": 1_148_161_000 + 6_258_176, "src": "f65eb04587b47385"},
@@ -55,7 +59,7 @@ NCU_TRAFFIC = {
 def kernel_source_hash() -> str:
     """Hash of the decode kernel's device code (the kernel whose traffic is quoted)."""
     h = hashlib.sha256()
-    for f in ("paged_decode_kernel.cuh", "pa_device.cuh"):
+    for f in ("paged_decode_kernel.cuh", "paged_merge.cuh", "pa_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_368_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -262,13 +266,180 @@ def run_reference(args):
 # ------------------------------------------------------------------ GPU arm
 
 
-def run_ours(args):
-    import ctypes
+LAUNCHES_PER_STEP = 2  # our kernels per step: reshape_and_cache_kernel + paged_decode_kernel
 
+
+class DecodeBench:
+    """One workload resident on the device, with the calls that time it."""
+
+    def __init__(self, lib, libpaged, wl, dev):
+        import torch
+
+        self.lib, self.wl, self.dev = lib, wl, dev
+        dt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+        self.dt = dt
+
+        def upload(raw):
+            return torch.from_numpy(np.ascontiguousarray(raw).view(np.int16).copy()).view(dt).to(dev)
+
+        shape = (wl.num_blocks, wl.num_kv_heads, wl.block_size, wl.head_dim)
+        self.k_cache = torch.zeros(shape, dtype=dt, device=dev)
+        self.v_cache = torch.zeros(shape, dtype=dt, device=dev)
+        idx = torch.from_numpy(wl.used).to(dev)
+        self.k_cache.index_copy_(0, idx, upload(wl.k_blocks))
+        self.v_cache.index_copy_(0, idx, upload(wl.v_blocks))
+        self.q, self.k_new, self.v_new = upload(wl.q), upload(wl.k_new), upload(wl.v_new)
+        self.slots = torch.from_numpy(wl.slot_mapping.astype(np.int64)).to(dev)
+        self.tables = torch.from_numpy(wl.block_tables.astype(np.int32)).to(dev)
+        self.ctx = torch.from_numpy(wl.context_lens.astype(np.int32)).to(dev)
+        self.out = torch.empty_like(self.q)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_ctx = wl.max_context_len
+        self.ws = libpaged.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, self.max_ctx,
+                                           device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        sp = self.stream.cuda_stream
+        kvh, D, bs, nb = wl.num_kv_heads, wl.head_dim, wl.block_size, wl.num_blocks
+        code = libpaged.dtype_code(dt)
+        mb = wl.max_blocks_per_seq
+        self.r_args = (self.k_new.data_ptr(), self.v_new.data_ptr(), self.k_cache.data_ptr(),
+                       self.v_cache.data_ptr(), self.slots.data_ptr(), wl.num_seqs, kvh, D, bs, nb, code,
+                       self.err.data_ptr(), sp)
+        self.d_args = (self.out.data_ptr(), self.q.data_ptr(), self.k_cache.data_ptr(), self.v_cache.data_ptr(),
+                       self.tables.data_ptr(), mb, self.ctx.data_ptr(), wl.num_seqs, self.max_ctx, float(wl.scale),
+                       wl.num_heads, kvh, D, bs, nb, code, self.ws.data_ptr(), self.ws.numel(), 0,
+                       self.err.data_ptr(), sp)
+        # end to end through the public API: one packed pinned host buffer of
+        # the step's inputs in, the result out (pa_decode_step_host)
+        offs, total = libpaged.step_inputs_layout(wl.num_seqs, wl.num_heads, kvh, D, mb)
+        self.h_in = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        t_ = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+        libpaged.pack_step_inputs(self.h_in, offs, q=t_(wl.q), key=t_(wl.k_new), value=t_(wl.v_new),
+                                  slot_mapping=t_(wl.slot_mapping.astype(np.int64)),
+                                  block_tables=t_(wl.block_tables.astype(np.int32)),
+                                  context_lens=t_(wl.context_lens.astype(np.int32)))
+        self.d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+        self.h_out = torch.empty(self.out.shape, dtype=dt).pin_memory()
+        self.h2d = total
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+        self.e_args = (self.h_in.data_ptr(), self.d_in.data_ptr(), self.h_out.data_ptr(), self.out.data_ptr(),
+                       self.k_cache.data_ptr(), self.v_cache.data_ptr(), wl.num_seqs, mb, self.max_ctx,
+                       float(wl.scale), wl.num_heads, kvh, D, bs, nb, code, self.ws.data_ptr(), self.ws.numel(),
+                       self.err.data_ptr(), sp)
+
+    def step(self):
+        st = self.lib.pa_reshape_and_cache(*self.r_args)
+        st |= self.lib.pa_decode(*self.d_args)
+        if st != 0:
+            raise SystemExit(f"libpaged call failed on {self.wl.name}")
+
+    def decode(self):
+        if self.lib.pa_decode(*self.d_args) != 0:
+            raise SystemExit(f"pa_decode failed on {self.wl.name}")
+
+    def e2e_step(self):
+        if self.lib.pa_decode_step_host(*self.e_args) != 0:
+            raise SystemExit(f"pa_decode_step_host failed on {self.wl.name}")
+
+    def check_flags(self):
+        import torch
+
+        torch.cuda.synchronize(self.dev)
+        if int(self.err.item()) != 0:
+            raise SystemExit(f"device error flags {int(self.err.item())} on {self.wl.name}")
+
+    # ---- timing helpers (CUDA events on the launching stream)
+
+    def time_back_to_back(self, fn, n):
+        """ms for n calls between one event pair (no events between the
+        launches, which would break the programmatic-launch overlap)."""
+        import torch
+
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(self.dev)
+        e0.record(self.stream)
+        for _ in range(n):
+            fn()
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return e0.elapsed_time(e1)
+
+    def time_each_decode(self, n, flush=None):
+        """Per-call ms of n pa_decode calls, an event pair around each (after
+        the step's append, so the cache is the step's); with `flush` a buffer
+        larger than L2 is rewritten before every call (cold L2)."""
+        import torch
+
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        torch.cuda.synchronize(self.dev)
+        for a, b in ev:
+            self.lib.pa_reshape_and_cache(*self.r_args)
+            if flush is not None:
+                flush.zero_()
+            a.record(self.stream)
+            self.decode()
+            b.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def calls_for(self, seconds, ms_per_call):
+        return int(max(1, seconds * 1e3 / max(ms_per_call, 1e-3)))
+
+
+def decode_summary(b, kvb, steps_ms, n_steps, per_call, cold, peak, e2e_ms, e2e_steps, unique=None):
+    mean = statistics.mean(per_call)
+    achieved = kvb / (mean * 1e-3) / 1e9
+    d = {"workload": describe(b.wl), "kv_bytes_per_step": kvb,
+         "step_us": steps_ms / n_steps * 1e3, "step_gbs": kvb * n_steps / (steps_ms * 1e-3) / 1e9,
+         "decode_us_mean": mean * 1e3, "decode_us_median": statistics.median(per_call) * 1e3,
+         "decode_us_min": min(per_call) * 1e3, "decode_calls": len(per_call),
+         "decode_gbs": achieved, "frac_of_measured_peak": achieved / peak, "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,
+         "decode_us_cold_l2_mean": statistics.mean(cold) * 1e3, "cold_l2_calls": len(cold),
+         "decode_gbs_cold_l2": kvb / (statistics.mean(cold) * 1e-3) / 1e9,
+         "e2e_gbs": kvb * e2e_steps / (e2e_ms * 1e-3) / 1e9, "e2e_us_per_step": e2e_ms / e2e_steps * 1e3}
+    d["frac_cold_l2_of_measured_peak"] = d["decode_gbs_cold_l2"] / peak
+    if unique is not None and unique != kvb:
+        d["unique_kv_bytes_per_step"] = unique
+        d["decode_gbs_unique"] = unique / (mean * 1e-3) / 1e9
+        d["frac_unique_of_measured_peak"] = d["decode_gbs_unique"] / peak
+        d["decode_gbs_unique_cold_l2"] = unique / (statistics.mean(cold) * 1e-3) / 1e9
+    return d
+
+
+def measure_config(lib, libpaged, wl, dev, peak, flush, seconds=0.5):
+    """Timings of one workload for the per-workload table: back-to-back steps
+    and per-call decode (each about `seconds` of device time), decode with a
+    flushed L2 before every call, and the end-to-end host step."""
+    import torch
+
+    b = DecodeBench(lib, libpaged, wl, dev)
+    for _ in range(5):
+        b.step()
+    b.check_flags()
+    one = b.time_back_to_back(b.step, 5) / 5
+    n = b.calls_for(seconds, one)
+    steps_ms = b.time_back_to_back(b.step, n)
+    per_call = b.time_each_decode(n)
+    cold = b.time_each_decode(min(200, n), flush=flush)
+    for _ in range(3):
+        b.e2e_step()
+    ne = max(20, n // 4)
+    e2e_ms = b.time_back_to_back(b.e2e_step, ne)
+    b.check_flags()
+    res = decode_summary(b, wl.kv_bytes(), steps_ms, n, per_call, cold, peak, e2e_ms, ne, wl.unique_kv_bytes())
+    del b
+    torch.cuda.empty_cache()
+    return res
+
+
+PER_CONFIG = [(2, None), (3, 8), (3, 16), (3, 32), (3, 64), (4, None), (0, None)]
+
+
+def run_ours(args):
     import torch
 
     from paged_kv_cache_368_b200 import build as pbuild
-    from paged_kv_cache_368_b200 import libpaged
+    from paged_kv_cache_368_b200 import inputs, libpaged
 
     world, rank, local = dist_init()
     if not torch.cuda.is_available():
@@ -284,136 +455,68 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     lib = libpaged.load()
+    dev = torch.device("cuda", local)
+    peak, peak_src = measured_peak()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     wl = load_workload(args)
-    dt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
-    dev = torch.device("cuda", local)
-
-    def upload(raw):
-        return torch.from_numpy(np.ascontiguousarray(raw).view(np.int16).copy()).view(dt).to(dev)
-
-    shape = (wl.num_blocks, wl.num_kv_heads, wl.block_size, wl.head_dim)
-    k_cache = torch.zeros(shape, dtype=dt, device=dev)
-    v_cache = torch.zeros(shape, dtype=dt, device=dev)
-    idx = torch.from_numpy(wl.used).to(dev)
-    k_cache.index_copy_(0, idx, upload(wl.k_blocks))
-    v_cache.index_copy_(0, idx, upload(wl.v_blocks))
-    q, k_new, v_new = upload(wl.q), upload(wl.k_new), upload(wl.v_new)
-    slots = torch.from_numpy(wl.slot_mapping.astype(np.int64)).to(dev)
-    tables = torch.from_numpy(wl.block_tables.astype(np.int32)).to(dev)
-    ctx = torch.from_numpy(wl.context_lens.astype(np.int32)).to(dev)
-    out = torch.empty_like(q)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    max_ctx = wl.max_context_len
-    ws = libpaged.alloc_workspace(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, max_ctx, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    sp = stream.cuda_stream
-    kvh, D, bs, nb = wl.num_kv_heads, wl.head_dim, wl.block_size, wl.num_blocks
-    code = libpaged.dtype_code(dt)
-    mb = wl.max_blocks_per_seq
-    r_args = (k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), slots.data_ptr(),
-              wl.num_seqs, kvh, D, bs, nb, code, err.data_ptr(), sp)
-    d_args = (out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), tables.data_ptr(), mb,
-              ctx.data_ptr(), wl.num_seqs, max_ctx, float(wl.scale), wl.num_heads, kvh, D, bs, nb, code,
-              ws.data_ptr(), ws.numel(), 0, err.data_ptr(), sp)
-
-    def step(dec_events=None):
-        st = lib.pa_reshape_and_cache(*r_args)
-        if dec_events is not None:
-            dec_events[0].record(stream)
-        st |= lib.pa_decode(*d_args)
-        if dec_events is not None:
-            dec_events[1].record(stream)
-        return st
-
+    b = DecodeBench(lib, libpaged, wl, dev)
     K, W = args.steps, args.warmup
     gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
     clocks = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
     time.sleep(0.3)
     for _ in range(W):
-        if step() != 0:
-            raise SystemExit("libpaged call failed in warm-up")
-    torch.cuda.synchronize(dev)
-    if int(err.item()) != 0:
-        raise SystemExit(f"device error flags {int(err.item())}")
+        b.step()
+    b.check_flags()
 
-    # ---- timed region 1: K whole steps, bracketed by one event pair (events
-    # between the launches would break the programmatic-launch overlap)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- timed region 1: exactly K whole steps, bracketed by a barrier and
+    # a synchronize, one event pair (max over ranks)
     if dist is not None:
         dist.barrier()
-    torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    e0.record(stream)
-    bad = 0
-    for i in range(K):
-        bad |= step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    elapsed_ms = reduce_max(b.time_back_to_back(b.step, K), dist, dev)
+
+    # ---- timed region 2 (roofline of the dominant kernel): an event pair
+    # around every pa_decode call, at least K calls and about 1 s of device
+    # time, so that the clock samples (every 100 ms) fall inside it
+    if dist is not None:
+        dist.barrier()
+    n_roof = max(K, b.calls_for(1.0, elapsed_ms / K))
+    dec_ms = b.time_each_decode(n_roof)
     t_wall1 = time.time()
-    if dist is not None:
-        dist.barrier()
-    if bad:
-        raise SystemExit("libpaged call failed in the timed region")
-    elapsed_ms = reduce_max(e0.elapsed_time(e1), dist, dev)
+    cold_ms = b.time_each_decode(min(200, n_roof), flush=flush)
 
-    # ---- timed region 2: the same steps with an event pair around every
-    # pa_decode call on its stream -> per-launch duration of the dominant kernel
-    dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    for i in range(K):
-        bad |= step(dec[i])
-    torch.cuda.synchronize(dev)
-    if bad:
-        raise SystemExit("libpaged call failed in the timed region")
-    dec_ms = [a.elapsed_time(b) for a, b in dec]
-
-    # ---- end to end through the public API: one packed pinned host buffer of
-    # the step's inputs in, the result out (pa_decode_step_host)
-    offs, total = libpaged.step_inputs_layout(wl.num_seqs, wl.num_heads, kvh, D, mb)
-    h_in = torch.zeros(total, dtype=torch.uint8).pin_memory()
-    t_ = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
-    libpaged.pack_step_inputs(h_in, offs, q=t_(wl.q), key=t_(wl.k_new), value=t_(wl.v_new),
-                              slot_mapping=t_(wl.slot_mapping.astype(np.int64)),
-                              block_tables=t_(wl.block_tables.astype(np.int32)),
-                              context_lens=t_(wl.context_lens.astype(np.int32)))
-    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
-    h_out = torch.empty(out.shape, dtype=dt).pin_memory()
-    h2d = total
-    d2h = h_out.numel() * h_out.element_size()
-    e_args = (h_in.data_ptr(), d_in.data_ptr(), h_out.data_ptr(), out.data_ptr(), k_cache.data_ptr(),
-              v_cache.data_ptr(), wl.num_seqs, mb, max_ctx, float(wl.scale), wl.num_heads, kvh, D, bs, nb, code,
-              ws.data_ptr(), ws.numel(), err.data_ptr(), sp)
-
-    def e2e_step():
-        if lib.pa_decode_step_host(*e_args) != 0:
-            raise SystemExit("pa_decode_step_host failed")
-
+    # ---- end to end through the public API (pa_decode_step_host)
     Ke = min(K, 2000)
     for _ in range(max(3, W)):
-        e2e_step()
-    torch.cuda.synchronize(dev)
+        b.e2e_step()
     if dist is not None:
         dist.barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(Ke):
-        e2e_step()
-    f1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = reduce_max(f0.elapsed_time(f1), dist, dev)
+    e2e_ms = reduce_max(b.time_back_to_back(b.e2e_step, Ke), dist, dev)
+    b.check_flags()
     clocks.stop()
 
     kvb = wl.kv_bytes()
     value = throughput_gbs(kvb, world, K, elapsed_ms)
-    mean_dec = statistics.mean(dec_ms)
-    achieved = kvb / (mean_dec * 1e-3) / 1e9
-    peak, peak_src = measured_peak()
+    head = decode_summary(b, kvb, elapsed_ms, K, dec_ms, cold_ms, peak, e2e_ms, Ke, wl.unique_kv_bytes())
     src = kernel_source_hash()
     tr = NCU_TRAFFIC.get(wl.name)
     traffic = tr["bytes"] if tr and tr.get("src") == src else None
+    h2d, d2h = b.h2d, b.d2h
+    del b
+    torch.cuda.empty_cache()
+
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = {}
+        for ci, bs in PER_CONFIG:
+            if ci == args.config and bs == args.block_size:
+                continue
+            w2 = inputs.config(ci, block_size=bs)
+            res = measure_config(lib, libpaged, w2, dev, peak, flush)
+            tr2 = NCU_TRAFFIC.get(w2.name)
+            res["traffic"] = tr2["bytes"] if tr2 and tr2.get("src") == src else None
+            per_config[w2.name] = res
 
     if rank != 0:
         if dist is not None:
@@ -427,20 +530,26 @@ def run_ours(args):
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": describe(wl), "kv_bytes_per_step": kvb, "unique_kv_bytes_per_step": wl.unique_kv_bytes(),
-                   "l2": f"inputs larger than L2 ({kvb / 2**20:.0f} MiB of KV per step vs 126 MiB L2); no flush",
-                   "parallelism": f"{world} independent replica(s), one per GPU", "step": "append + decode + merge"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "pa_decode (decode + merge launches)",
-                     "timing": "CUDA events around each pa_decode call in a second pass over the K steps",
-                     "peak_source": peak_src, "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,
-                     "decode_us_mean": mean_dec * 1e3, "decode_us_median": statistics.median(dec_ms) * 1e3,
-                     "decode_us_min": min(dec_ms) * 1e3, "kernel_src": src},
+                   "l2": (f"inputs larger than L2 ({kvb / 2**20:.0f} MiB of KV per step vs 126 MiB L2), no flush "
+                          "between timed steps; decode_us_cold_l2 flushes a 252 MiB buffer before every call"),
+                   "parallelism": f"{world} independent replica(s), one per GPU",
+                   "step": "append (pa_reshape_and_cache) + decode with in-launch merge (pa_decode)"},
+        "roofline": {"bound": "hbm", "achieved": head["decode_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": head["decode_gbs"] / peak, "traffic": traffic,
+                     "kernel": "paged_decode_kernel (pa_decode: one launch, merge included)",
+                     "timing": (f"CUDA events around each of {len(dec_ms)} pa_decode calls (>= 1 s of device time) "
+                                "on the launching stream, after the step's append"),
+                     "peak_source": peak_src, "frac_of_8tbs_spec": head["decode_gbs"] / SPEC_HBM_GBS,
+                     "decode_us_mean": head["decode_us_mean"], "decode_us_median": head["decode_us_median"],
+                     "decode_us_min": head["decode_us_min"], "decode_us_cold_l2_mean": head["decode_us_cold_l2_mean"],
+                     "frac_cold_l2": head["frac_cold_l2_of_measured_peak"], "kernel_src": src},
         "cpu_baseline": cpu,
         "e2e": {"value": throughput_gbs(kvb, world, Ke, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke, "ms_per_step": e2e_ms / Ke,
                 "path": "pa_decode_step_host (C ABI): packed pinned host inputs -> device (1 copy), append, decode, output -> pinned host (1 copy)"},
-        "gpu_launches": 3 * K,
+        "gpu_launches": LAUNCHES_PER_STEP * K,
         "clocks": clocks.summary(t_wall0, t_wall1),
+        "per_config": per_config,
     }
     print(json.dumps(line), flush=True)
     if dist is not None:
@@ -662,6 +771,8 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (1 = LLaMA-7B-shaped layer)")
     ap.add_argument("--block-size", type=int, default=None, help="block size for workload 3 (LLaMA-13B)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload table (all five workloads, LLaMA-13B at block sizes 8-64)")
     ap.add_argument("--op", choices=("step", "block_ops", "prefill"), default="step",
                     help="step: the decode step (default); block_ops: block copy/swap throughput; "
                          "prefill: multi-token causal paged attention")

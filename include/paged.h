@@ -90,8 +90,10 @@ PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, void* 
 
 /*
  * Bytes of device workspace pa_decode needs on the CURRENT device for this
- * shape (it depends on the device's SM count, not on the context lengths).
- * Returns 0 for invalid or unsupported arguments.
+ * shape with the largest grid (one CTA per SM; it depends on the device's SM
+ * count, not on the context lengths).  A call with max_ctas > 0 needs less:
+ * the workspace of a grid of n CTAs is enough for it.  Returns 0 for invalid
+ * or unsupported arguments.
  */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                 int max_context_len);
@@ -104,16 +106,27 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_h
  * anything.  context_lens[s] == 0 writes zeros.  Accumulation is fp32; the
  * result is rounded to `dtype`.
  *
+ * One kernel launch: every (sequence, kv-head) context is cut into 16-token
+ * chunks that are spread evenly over a persistent grid; a context split
+ * across warps is merged by log-sum-exp inside the same launch (the last
+ * warp to finish its part merges; no warp waits for another).
+ *
  * max_context_len: an upper bound on context_lens (used to size the launch).
- * workspace: device buffer of at least pa_decode_workspace_size() bytes,
- *   16-byte aligned, owned by the caller; its contents need no
- *   initialisation and are scratch after the call.  Calls that overlap on the
+ * workspace: device buffer, 16-byte aligned, owned by the caller, of at
+ *   least pa_decode_workspace_size() bytes (or the size for the capped grid
+ *   when max_ctas > 0; PA_ERR_WORKSPACE if smaller).  It must be ZERO-FILLED
+ *   before its first use (cudaMemset once): it holds the merge's ticket
+ *   counters, which every call leaves at zero again, also when a wait gave
+ *   up (PA_ERRF_TIMEOUT).  The rest is scratch.  Calls that overlap on the
  *   GPU must use different workspaces.
  * max_ctas: 0 = one CTA per SM (default); n > 0 caps the grid at n CTAs
  *   (fewer, longer per-warp runs -> fewer split partitions).  The result is
  *   the same attention for every choice, up to fp32 rounding order.
  * Supported: head_dim in {64, 128}; block_size in {8, 16, 32, 64};
- *   num_heads/num_kv_heads in {1, 2, 4, 8}; 1 <= num_seqs <= 2048;
+ *   num_heads/num_kv_heads in {1, 2, 4, 8}; 1 <= num_seqs <= 16384 while
+ *   the per-sequence prefix table (4 bytes a sequence) fits in shared memory
+ *   beside the pipeline stages (PA_ERR_UNSUPPORTED otherwise);
+ *   num_kv_heads < 32768;
  *   num_seqs * num_kv_heads * ceil(max_context_len/16) < 2^31.
  */
 PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -152,21 +165,30 @@ PA_API pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, void*
 
 /*
  * pa_decode_static -- pa_decode for callers that cannot allocate device
- * memory (code where cudaMalloc is not allowed or not available, such as a
- * host callback, a thread that must never block on an allocator, or a host
- * application that hands a plugin only its input and output buffers).  The
- * pages have no counterpart of this entry point; it exists for such callers.
+ * memory: a plugin whose host application owns every device allocation and
+ * hands it only input and output buffers, code under an allocation policy
+ * that forbids cudaMalloc on its path (a thread that must never block on an
+ * allocator, a fixed memory budget), or a binding with no device allocator.
+ * The pages have no counterpart of this entry point; it exists for such
+ * callers.  It enqueues kernels, so call it from an ordinary host thread
+ * (never from a host function enqueued on a stream, where CUDA calls are
+ * not allowed).
  *
  * Same arguments and result as pa_decode, minus the workspace: the scratch
  * is a 10 MiB array inside the library's device image, reserved on every
- * GPU that uses this call until the process exits.  A shape that needs more
- * scratch than that (pa_decode_workspace_size) returns PA_ERR_WORKSPACE; on
- * a 148-SM B200 every supported shape fits.  All calls on one GPU share the
- * array: calls that can run at the same time on that GPU race and give wrong
- * results, so serialise them.  The array needs no clearing between calls.
- * The first call on a device looks up the array's address
- * (cudaGetSymbolAddress); make it before any stream capture on that device.
- * Nothing is allocated or freed.
+ * GPU where the library's module is loaded, until the process exits.  The
+ * scratch a call needs is that of the grid it launches: every supported
+ * shape fits on a GPU of up to 148 SMs (a B200); on a larger GPU a shape
+ * that does not fit returns PA_ERR_WORKSPACE (see pa_last_error), and
+ * max_ctas > 0 shrinks the grid and its scratch.  Argument errors return
+ * PA_ERR_INVALID / PA_ERR_UNSUPPORTED before any CUDA call.  All calls on one
+ * GPU share the array, which keeps what the last call left: calls that can
+ * run at the same time on that GPU race and give wrong results, so
+ * serialise them.  The first call in a CUDA context sets the array up: it
+ * looks up its device address (cudaGetSymbolAddress) and zeroes the merge's
+ * ticket counters with cudaMemsetAsync on `stream` (every call leaves them
+ * at zero again).  Make that first call before any stream capture on that
+ * device.  Nothing is allocated or freed.
  */
 PA_API pa_status pa_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
                            const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,

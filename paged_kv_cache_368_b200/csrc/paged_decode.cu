@@ -19,8 +19,11 @@
 //    chunk and no partition-size heuristic is needed.
 //  * A warp's run is cut at unit boundaries into segments.  A segment that
 //    covers a whole unit writes the normalised output directly; a unit split
-//    across warps leaves un-normalised partials (m, l, o) that the merge
-//    kernel combines by log-sum-exp.
+//    across warps leaves un-normalised partials (m, l, o), and each
+//    contributing warp then adds its chunk count to the unit's ticket
+//    counter.  The warp that completes the count merges the partials by
+//    log-sum-exp and writes the output, in the same launch: no warp waits
+//    for another and there is no second kernel.
 //  * Each warp is its own producer: lane 0 issues TMA tile loads (128-byte
 //    swizzle, L2 evict-first) of the K and V rows of chunk k+DEPTH into a
 //    per-warp ring of shared-memory stages, completion counted on an
@@ -40,26 +43,11 @@
 #include <mutex>
 
 #include "paged_decode_kernel.cuh"
-#include "paged_merge.cuh"
 #include "pa_host.h"
 
 // =============================================================== host side
 
 namespace {
-
-struct WsLayout {
-  size_t header, jobs, ml, o, total;
-};
-
-WsLayout ws_layout(int max_warps, int G, int D) {
-  WsLayout w;
-  w.header = 0;
-  w.jobs = 256;
-  w.ml = w.jobs + (size_t(max_warps) * 16 + 255) / 256 * 256;
-  w.o = w.ml + (size_t(2) * max_warps * G * 8 + 255) / 256 * 256;
-  w.total = w.o + size_t(2) * max_warps * G * D * 4;
-  return w;
-}
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -157,13 +145,6 @@ pa_status launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pa::
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, p);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_kernel", e);
-  // One CTA per warp of the decode grid (each may own a merge job).
-  cudaLaunchConfig_t mcfg = cfg;
-  mcfg.gridDim = dim3(p.total_warps);
-  mcfg.blockDim = dim3(pa::merge_threads(D, G));
-  mcfg.dynamicSmemBytes = size_t(p.total_warps) * sizeof(int);
-  e = cudaLaunchKernelEx(&mcfg, pa::paged_decode_merge_kernel<T, D, G>, p);
-  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "launching paged_decode_merge_kernel", e);
   return PA_OK;
 }
 
@@ -183,6 +164,56 @@ bool valid_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 
 
 }  // namespace
 
+namespace pa {
+
+// Host checks of a decode call's sizes (no CUDA call).  Returns PA_OK and
+// fills the shape part of `plan`, or the status to return without launching.
+pa_status plan_decode(int num_seqs, int max_blocks_per_seq, int max_context_len, float scale, int num_heads,
+                      int num_kv_heads, int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                      int max_ctas, DecodePlan* plan) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return PA_ERR_INVALID;
+  if (max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0 || max_ctas < 0) return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID;
+  const int G = num_heads / num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!valid_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > kMaxSeqs || num_kv_heads >= (1 << 15)) return PA_ERR_UNSUPPORTED;
+  const int64_t cap64 = std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * block_size);
+  const int64_t upper = (int64_t)num_seqs * num_kv_heads * ((cap64 + kChunk - 1) / kChunk);
+  if (upper >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  if (num_blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  plan->G = G;
+  plan->head_dim = head_dim;
+  plan->ctx_cap = static_cast<int>(cap64);
+  plan->warps = warps_for(head_dim, G);
+  plan->ctas = 0;
+  plan->layout = ws_layout(0, G, head_dim);
+  plan->upper_chunks = upper;
+  return PA_OK;
+}
+
+// The grid for the current device (its SM count) and its workspace layout.
+pa_status plan_decode_grid(int max_ctas, DecodePlan* plan) {
+  const int64_t upper = plan->upper_chunks;
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice", ce);
+  const int sms = device_sms(dev);
+  if (sms <= 0) return fail(PA_ERR_CUDA, "querying the SM count", cudaSuccess);
+  // A persistent grid: at most one CTA per SM, and no more CTAs than give
+  // each warp about four chunks.
+  int ctas = static_cast<int>(std::min<int64_t>(sms, std::max<int64_t>(1, (upper + plan->warps * 4 - 1) /
+                                                                            (plan->warps * 4))));
+  if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
+  plan->ctas = ctas;
+  plan->layout = ws_layout(ctas * plan->warps, plan->G, plan->head_dim);
+  return PA_OK;
+}
+
+}  // namespace pa
+
 extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                            int max_context_len) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return 0;
@@ -194,7 +225,8 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   const int sms = pa::device_sms(dev);
   if (sms <= 0) return 0;
-  return ws_layout(sms * pa::warps_for(head_dim, G), G, head_dim).total;
+  // The largest grid this shape can launch on this device (one CTA per SM).
+  return pa::ws_layout(sms * pa::warps_for(head_dim, G), G, head_dim).total;
 }
 
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -202,37 +234,20 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
                                int num_seqs, int max_context_len, float scale, int num_heads, int num_kv_heads,
                                int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype, void* workspace,
                                size_t workspace_bytes, int max_ctas, int32_t* err_flags, pa_stream_t stream) {
-  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return PA_ERR_INVALID;
-  if (max_blocks_per_seq <= 0 || max_context_len < 0 || num_blocks <= 0 || max_ctas < 0) return PA_ERR_INVALID;
-  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID;
-  if (!std::isfinite(scale)) return PA_ERR_INVALID;
-  const int G = num_heads / num_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
-  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (!valid_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-  if (num_seqs > pa::kMaxSeqs || num_kv_heads >= (1 << 15)) return PA_ERR_UNSUPPORTED;
+  pa::DecodePlan plan;
+  const pa_status st = pa::plan_decode(num_seqs, max_blocks_per_seq, max_context_len, scale, num_heads,
+                                       num_kv_heads, head_dim, block_size, num_blocks, dtype, max_ctas, &plan);
+  if (st != PA_OK) return st;
   if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID;
-  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(block_tables, 4) || !aligned(context_lens, 4))
-    return PA_ERR_INVALID;
-  const int64_t cap64 = std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * block_size);
-  const int ctx_cap = static_cast<int>(cap64);
-  const int64_t upper = (int64_t)num_seqs * num_kv_heads * ((cap64 + pa::kChunk - 1) / pa::kChunk);
-  if (upper >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
-  if (num_blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-
+  if (!pa::decode_pointers_ok(out, q, k_cache, v_cache, block_tables, context_lens)) return PA_ERR_INVALID;
+  const pa_status gst = pa::plan_decode_grid(max_ctas, &plan);
+  if (gst != PA_OK) return gst;
+  const pa::WsLayout& L = plan.layout;
+  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return PA_ERR_WORKSPACE;
+  const int G = plan.G, ctas = plan.ctas, warps = plan.warps;
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
   if (ce != cudaSuccess) return pa::fail(PA_ERR_CUDA, "cudaGetDevice", ce);
-  const int sms = pa::device_sms(dev);
-  if (sms <= 0) return pa::fail(PA_ERR_CUDA, "querying the SM count", cudaSuccess);
-  const int warps = pa::warps_for(head_dim, G);
-  const WsLayout L = ws_layout(sms * warps, G, head_dim);
-  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 16)) return PA_ERR_WORKSPACE;
-
-  int ctas = static_cast<int>(std::min<int64_t>(sms, std::max<int64_t>(1, (upper + warps * 4 - 1) / (warps * 4))));
-  if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
 
   CUtensorMap km, vm;
   if (!pa::have_tensor_map_encoder())
@@ -247,15 +262,14 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   p.q = q;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  p.ws_header = reinterpret_cast<int*>(ws + L.header);
-  p.ws_jobs = reinterpret_cast<int4*>(ws + L.jobs);
+  p.ws_tickets = reinterpret_cast<int*>(ws + L.tickets);
   p.ws_ml = reinterpret_cast<float2*>(ws + L.ml);
   p.ws_o = reinterpret_cast<float*>(ws + L.o);
   p.err_flags = err_flags;
   p.num_blocks = num_blocks;
   p.num_seqs = num_seqs;
   p.max_blocks_per_seq = max_blocks_per_seq;
-  p.ctx_cap = ctx_cap;
+  p.ctx_cap = plan.ctx_cap;
   p.max_context_len = max_context_len;
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;

@@ -5,11 +5,12 @@
 #include <type_traits>
 
 #include "pa_device.cuh"
+#include "paged_merge.cuh"
 
 namespace pa {
 
 constexpr int kChunk = 16;       // tokens per pipeline stage
-constexpr int kMaxSeqs = 2048;   // prefix table lives in shared memory
+constexpr int kMaxSeqs = 16384;  // prefix table lives in shared memory (4 bytes a sequence)
 #ifndef PA_CORE_WARPS
 #define PA_CORE_WARPS 8
 #endif
@@ -44,8 +45,9 @@ struct DecodeParams {
   const int32_t* context_lens;
   float* ws_o;       // [2W][G][D] un-normalised partial outputs
   float2* ws_ml;     // [2W][G] (running max in log2 units, running sum)
-  int4* ws_jobs;     // [W] merge jobs
-  int* ws_header;    // [0] = total chunks
+  int* ws_tickets;   // [W] chunks of a split unit accounted for so far, indexed
+                     // by the warp holding the unit's first chunk; every
+                     // launch leaves them at zero (callers zero them once)
   int32_t* err_flags;
   int64_t num_blocks;
   int num_seqs;
@@ -87,28 +89,41 @@ struct ChunkRaw {
   int ctx, p0, p1;
 };
 
-__device__ __forceinline__ ChunkRaw chunk_load(const DecodeParams& p, const int* prefix, int64_t g, int64_t end) {
-  ChunkRaw r;
-  r.seq = -1;
-  r.head = r.c = r.nc = r.ctx = r.p0 = 0;
-  r.p1 = -1;
-  if (g >= end) return r;
+// Unit (sequence, kv-head) of global chunk g < KVH * prefix[S], the chunk's
+// index c in it and the unit's chunk count nc (shared-memory lookups only).
+struct UnitPos {
+  int seq, head, c, nc;
+};
+
+__device__ __forceinline__ UnitPos unit_pos(const DecodeParams& p, const int* prefix, int64_t g) {
   const int KVH = p.num_kv_heads;
   int lo = 0, hi = p.num_seqs;  // largest s in [0, S) with KVH*prefix[s] <= g
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if ((int64_t)KVH * prefix[mid] <= g) lo = mid; else hi = mid;
   }
-  const int s = lo;
-  const int nc = prefix[s + 1] - prefix[s];
-  const int rem = static_cast<int>(g - (int64_t)KVH * prefix[s]);
-  const int h = rem / nc;
-  const int c = rem - h * nc;
+  UnitPos u;
+  u.seq = lo;
+  u.nc = prefix[lo + 1] - prefix[lo];
+  const int rem = static_cast<int>(g - (int64_t)KVH * prefix[lo]);
+  u.head = rem / u.nc;
+  u.c = rem - u.head * u.nc;
+  return u;
+}
+
+__device__ __forceinline__ ChunkRaw chunk_load(const DecodeParams& p, const int* prefix, int64_t g, int64_t end) {
+  ChunkRaw r;
+  r.seq = -1;
+  r.head = r.c = r.nc = r.ctx = r.p0 = 0;
+  r.p1 = -1;
+  if (g >= end) return r;
+  const UnitPos u = unit_pos(p, prefix, g);
+  const int s = u.seq, c = u.c;
   const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
   r.seq = s;
-  r.head = h;
+  r.head = u.head;
   r.c = c;
-  r.nc = nc;
+  r.nc = u.nc;
   r.ctx = __ldg(p.context_lens + s);
   if (p.block_size >= kChunk) {
     r.p0 = __ldg(row + c * kChunk / p.block_size);
@@ -535,8 +550,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
 
   const int S = p.num_seqs, H = p.num_heads;
   const int64_t NC = (int64_t)p.num_kv_heads * prefix[S];
-  if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_header[0] = static_cast<int>(NC);
-  const int64_t c0 = (int64_t)gw * NC / W, c1 = (int64_t)(gw + 1) * NC / W;
+  const int64_t c0 = run_begin(gw, NC, W), c1 = run_begin(gw + 1, NC, W);
   const int n = static_cast<int>(c1 - c0);
 
   // Chunk windows: `cur` holds chunks [kb, kb+32), `nxt` [kb+32, kb+64), and
@@ -603,7 +617,6 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
   st.reset();
   bool seg_from_unit_start = false;
   bool first_seg = true;
-  bool job_written = false;
   bool timed_out = false;
   int k = 0;
   for (; k < n; ++k) {
@@ -658,21 +671,6 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
         const int slot = 2 * gw + (first_seg ? 0 : 1);
         st.write_partial(p.ws_o + (int64_t)slot * G * D, p.ws_ml + (int64_t)slot * G, lane);
       }
-      if (k == n - 1) {
-        // The unit this warp's run ends in started here and continues in the
-        // next warps: this warp owns its merge job.
-        const int c = __shfl_sync(kFull, cur.c, d);
-        const int nc = __shfl_sync(kFull, cur.nc, d);
-        if (lane == 0) {
-          if (seg_from_unit_start && !unit_end) {
-            const int64_t a = c0 + k - c;
-            p.ws_jobs[gw] = make_int4(seq, kvh, static_cast<int>(a), nc);
-          } else {
-            p.ws_jobs[gw] = make_int4(-1, 0, 0, 0);
-          }
-        }
-        job_written = true;
-      }
       first_seg = false;
     }
   }
@@ -682,7 +680,40 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     for (int kk = k; kk < n && kk < k + DEPTH; ++kk)
       mbar_wait_bounded(&bars[warp * DEPTH + (kk % DEPTH)], (kk / DEPTH) & 1, kWaitLimitNs);
   }
-  if (!job_written && lane == 0) p.ws_jobs[gw] = make_int4(-1, 0, 0, 0);
+  if (n == 0) return;
+
+  // Split units: the run's first and last segments may each cover only part
+  // of a unit.  For each such part the warp adds its chunk count to the
+  // unit's ticket counter; the warp whose addition completes the unit's
+  // count merges every part and writes the output, so no warp ever waits
+  // for another.  Tickets are taken after the run (also when a wait gave
+  // up, so the counters always return to zero; the outputs are then flagged
+  // as not written).
+  const UnitPos uf = unit_pos(p, prefix, c0), ul = unit_pos(p, prefix, c1 - 1);
+  const int64_t af = c0 - uf.c, al = c1 - 1 - ul.c;  // global first chunks of the two units
+  auto take_ticket = [&](int64_t a, const UnitPos& u, int mine) {
+    __threadfence();  // this lane's partial stores before the ticket
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      int* t = p.ws_tickets + warp_of_chunk(a, NC, W);
+      const int before = atomicAdd(t, mine);
+      last = before + mine == u.nc;
+      if (last) *t = 0;  // all parts counted; nobody else touches it in this launch
+    }
+    if (__shfl_sync(kFull, last, 0)) {
+      __threadfence();  // the other parts' stores, published before their tickets
+      merge_split_unit<T, D, G>(p.ws_ml, p.ws_o,
+                                static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D, a,
+                                u.nc, NC, W, lane);
+    }
+  };
+  if (af == al) {  // the whole run lies in one unit
+    if (!(uf.c == 0 && ul.c == ul.nc - 1)) take_ticket(af, uf, n);
+  } else {
+    if (uf.c != 0) take_ticket(af, uf, uf.nc - uf.c);
+    if (ul.c != ul.nc - 1) take_ticket(al, ul, ul.c + 1);
+  }
 }
 
 }  // namespace pa

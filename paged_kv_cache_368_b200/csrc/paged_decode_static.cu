@@ -2,42 +2,68 @@
 // device memory.
 //
 // pa_decode needs a caller-provided workspace for the partial results of
-// units split across warps.  Some callers have no way to provide one: code
-// running where cudaMalloc is forbidden or unavailable (for example inside a
-// host callback, a real-time thread that must not block on the allocator,
-// or a plugin host that owns every device allocation and hands out only
-// input/output buffers).  For them this entry point uses a scratch area that
-// is part of the library image itself: a fixed-size array in device global
-// memory, reserved when the library's module is loaded on a GPU.
+// units split across warps.  Some callers have no way to provide one: a
+// plugin whose host application owns every device allocation and hands it
+// only input and output buffers, code running under an allocation policy
+// that forbids cudaMalloc on its path (a real-time thread that must never
+// block on the allocator, a pre-planned memory budget), or a binding that
+// has no device allocator at all.  For them this entry point uses a scratch
+// area that is part of the library image itself: a fixed-size array in
+// device global memory, reserved when the library's module is loaded on a
+// GPU.  The call enqueues kernels (and, the first time on a device, a memset
+// of the array's counters), so it must run on an ordinary host thread, never
+// inside a host function enqueued on a stream, where CUDA calls are not
+// allowed.
 //
 // Properties a user must know:
-//  * The scratch holds kStaticScratchBytes (10 MiB).  Every GPU on which this
-//    entry point is used keeps that memory reserved until the process exits.
-//    The shapes the library supports need at most 9.5 MiB on a 148-SM B200;
-//    a request that needs more (a GPU with more SMs) is rejected with
-//    PA_ERR_WORKSPACE and a pa_last_error() message -- pass max_ctas to
-//    shrink the grid (and the scratch it needs) in that case.
+//  * The scratch holds kStaticScratchBytes (10 MiB).  Every GPU on which the
+//    library's module is loaded keeps that memory reserved until the process
+//    exits.  The need is computed for the grid that will actually be
+//    launched (pa_decode's plan): every supported shape fits on a GPU of up
+//    to 148 SMs (checked at compile time below); on a larger GPU a shape that
+//    does not fit is rejected with PA_ERR_WORKSPACE and a pa_last_error()
+//    message, and passing max_ctas > 0 shrinks the grid, and the scratch it
+//    needs, until it fits.
 //  * All calls share the one array per GPU.  Calls whose kernels may run at
 //    the same time on one GPU (different streams, different host threads)
 //    race on it and produce wrong results: serialise them.
-//  * The kernel writes every scratch word before reading it in the same
-//    call, so nothing has to start at zero and the contents a previous call
-//    left behind are harmless.
+//  * The array keeps what the last call left.  The only words that must start
+//    at zero are the split-unit ticket counters, which every decode launch
+//    returns to zero; they are cleared once, when the array is first set up
+//    on a device (a cudaMemsetAsync on the caller's stream).
 //  * The first call on a device looks up the array's device address with
-//    cudaGetSymbolAddress (which may load the module).  Make that first call
-//    before any stream capture begins on that device.
+//    cudaGetSymbolAddress (which may load the module) and clears the
+//    counters.  Make that first call before any stream capture begins on
+//    that device.  The address is cached per CUDA context; after
+//    cudaDeviceReset the first call in the new context sets up again.
 //  * No device memory is allocated or freed: no cudaMalloc/cudaFree and no
 //    allocating library routine is called.
-#include <atomic>
 #include <cstdio>
 #include <mutex>
 
 #include "pa_device.cuh"
+#include "pa_host.h"
+#include "paged_decode_kernel.cuh"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(10) << 20;
-constexpr int kMaxDevices = 64;
+constexpr int kLargestGridSMs = 148;  // B200
+
+constexpr size_t largest_need(int sms) {
+  size_t need = 0;
+  for (int D : {64, 128})
+    for (int G : {1, 2, 4, 8}) {
+      const size_t n = pa::ws_layout(sms * pa::warps_for(D, G), G, D).total;
+      need = n > need ? n : need;
+    }
+  return need;
+}
+static_assert(largest_need(kLargestGridSMs) <= kStaticScratchBytes,
+              "the static scratch must hold the workspace of every supported shape on a 148-SM GPU");
+
+// Ticket counters of the largest grid any shape can launch on `sms` SMs.
+size_t ticket_bytes(int sms) { return pa::ws_layout(sms * 8, 1, 64).ml; }
 
 }  // namespace
 
@@ -45,28 +71,69 @@ static __device__ __align__(256) unsigned char pa_static_scratch[kStaticScratchB
 
 namespace {
 
-// Device address of pa_static_scratch on device `dev` (the current device),
-// looked up once per device.  The host-side name of the array is only a
-// stand-in: a kernel must be given this address, never &pa_static_scratch.
-void* static_scratch_address(int dev, cudaError_t* err) {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  return fn;
+}
+
+// Device address of pa_static_scratch in the current context, set up once per
+// context: the address is looked up (the host-side name of the array is only
+// a stand-in, never a device address) and the ticket counters are zeroed on
+// `stream`.
+void* static_scratch_address(int dev, cudaStream_t stream, cudaError_t* err, const char** what) {
   static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
+  static CUcontext ctx_of[pa::kMaxDevices * 2] = {};
+  static void* addr_of[pa::kMaxDevices * 2] = {};
   *err = cudaSuccess;
-  if (dev < 0 || dev >= kMaxDevices) {
-    *err = cudaErrorInvalidDevice;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) {
+    *err = cudaErrorNotSupported;
+    *what = "pa_decode_static: cuCtxGetCurrent entry point not found";
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, pa_static_scratch);
-    if (e != cudaSuccess) {
-      *err = e;
-      return nullptr;
-    }
-    addr[dev] = p;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) == CUDA_SUCCESS && ctx != nullptr)
+    for (int i = 0; i < pa::kMaxDevices * 2; ++i)
+      if (ctx_of[i] == ctx) return addr_of[i];
+  // Not set up in this context yet.  The lookup also creates the device's
+  // primary context if no context is current.
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, pa_static_scratch);
+  if (e != cudaSuccess) {
+    *err = e;
+    *what = "pa_decode_static: cudaGetSymbolAddress";
+    return nullptr;
   }
-  return addr[dev];
+  if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+    *err = cudaErrorInvalidDevice;
+    *what = "pa_decode_static: cuCtxGetCurrent";
+    return nullptr;
+  }
+  const int sms = pa::device_sms(dev);
+  e = cudaMemsetAsync(p, 0, ticket_bytes(sms), stream);
+  if (e != cudaSuccess) {
+    *err = e;
+    *what = "pa_decode_static: clearing the ticket counters";
+    return nullptr;
+  }
+  for (int i = 0; i < pa::kMaxDevices * 2; ++i)
+    if (ctx_of[i] == nullptr) {
+      ctx_of[i] = ctx;
+      addr_of[i] = p;
+      break;
+    }
+  return p;
 }
 
 }  // namespace
@@ -77,18 +144,28 @@ extern "C" pa_status pa_decode_static(void* out, const void* q, const void* k_ca
                                       int num_heads, int num_kv_heads, int head_dim, int block_size,
                                       int64_t num_blocks, pa_dtype dtype, int max_ctas, int32_t* err_flags,
                                       pa_stream_t stream) {
+  pa::DecodePlan plan;
+  const pa_status st = pa::plan_decode(num_seqs, max_blocks_per_seq, max_context_len, scale, num_heads,
+                                       num_kv_heads, head_dim, block_size, num_blocks, dtype, max_ctas, &plan);
+  if (st != PA_OK) return st;
+  if (num_seqs == 0) return PA_OK;
+  if (!pa::decode_pointers_ok(out, q, k_cache, v_cache, block_tables, context_lens)) return PA_ERR_INVALID;
+  const pa_status gst = pa::plan_decode_grid(max_ctas, &plan);
+  if (gst != PA_OK) return gst;
+  if (plan.layout.total > kStaticScratchBytes) {
+    char msg[200];
+    snprintf(msg, sizeof(msg),
+             "pa_decode_static: a %d-CTA grid needs %zu bytes of scratch, the static area holds %zu "
+             "(pass max_ctas to shrink the grid)",
+             plan.ctas, plan.layout.total, kStaticScratchBytes);
+    return pa::fail(PA_ERR_WORKSPACE, msg, cudaSuccess);
+  }
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_static: cudaGetDevice", e);
-  const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len);
-  if (need > kStaticScratchBytes) {
-    char msg[160];
-    snprintf(msg, sizeof(msg), "pa_decode_static: needs %zu bytes of scratch, the static area holds %zu", need,
-             kStaticScratchBytes);
-    return pa::fail(PA_ERR_WORKSPACE, msg, cudaSuccess);
-  }
-  void* scratch = static_scratch_address(dev, &e);
-  if (scratch == nullptr) return pa::fail(PA_ERR_CUDA, "pa_decode_static: cudaGetSymbolAddress", e);
+  const char* what = "";
+  void* scratch = static_scratch_address(dev, reinterpret_cast<cudaStream_t>(stream), &e, &what);
+  if (scratch == nullptr) return pa::fail(PA_ERR_CUDA, what, e);
   return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                    max_context_len, scale, num_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype, scratch,
                    kStaticScratchBytes, max_ctas, err_flags, stream);

@@ -1,17 +1,35 @@
-// LSE merge of the partials of units split across warps (device code).
+// Log-sum-exp merge of a unit split across warps, run inside the decode
+// kernel by the last warp to finish its part of the unit (device code).
+//
+// A (sequence, kv-head) unit whose chunks span several warps' runs leaves one
+// un-normalised partial (m, l, o) per contributing warp, m in log2 units:
+//   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
+// ("【infra之路】10-PagedAttention 与 KV Cache 管理", section 8 Q2: FlashDecoding
+// splits a long context and combines the pieces; this is that combination).
 #pragma once
 
-#include "paged_decode_kernel.cuh"
+#include "pa_device.cuh"
 
 namespace pa {
 
-// --------------------------------------------------------------- merge kernel
+// The global chunk order is split evenly over W warps: warp w runs chunks
+// [floor(w*NC/W), floor((w+1)*NC/W)).
+__device__ __forceinline__ int64_t run_begin(int64_t w, int64_t NC, int W) { return w * NC / W; }
 
-// Threads of one merge CTA: enough that every (q-head, 4 columns) item has
-// several threads sharing out the contributors.
-__host__ __device__ constexpr int merge_threads(int D, int G) { return G * D / 4 >= 256 ? 1024 : 256; }
+// The warp whose run holds global chunk g: the w with
+// floor(w*NC/W) <= g < floor((w+1)*NC/W), i.e. ceil((g+1)*W/NC) - 1.
+__device__ __forceinline__ int warp_of_chunk(int64_t g, int64_t NC, int W) {
+  return static_cast<int>(((g + 1) * W + NC - 1) / NC - 1);
+}
 
-// One online-softmax fold of a partial (ml, o) into the running (m, l, acc).
+// Partial slot of warp w's part of the unit that starts at global chunk a:
+// slot 2w holds a warp's first segment, slot 2w+1 its last.  The part is the
+// warp's first segment exactly when its run starts at or after a.
+__device__ __forceinline__ int64_t partial_slot(int64_t w, int64_t a, int64_t NC, int W) {
+  return 2 * w + (run_begin(w, NC, W) >= a ? 0 : 1);
+}
+
+// One online-softmax fold of a partial (ml = (m, l), o) into (m, l, acc).
 __device__ __forceinline__ void fold_partial(float& m, float& l, float4& acc, float2 ml, float4 o) {
   const float mn = fmaxf(m, ml.x);
   const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
@@ -23,85 +41,71 @@ __device__ __forceinline__ void fold_partial(float& m, float& l, float4& acc, fl
   m = mn;
 }
 
-// Combines the partials of a unit split across warps w0..w1:
-//   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
-// (m in log2 units).  One CTA per merge job.  The contributors' partial
-// slots are resolved once into shared memory; thread (group, item) then folds
-// contributors j = group, group + NGRP, ... of one (q-head, 4 columns) item
-// into a running (m, l, acc), loading four contributors at a time, and the
-// NGRP groups are combined once through shared memory.
+// Merge the partials of the unit of `nc` chunks starting at global chunk `a`
+// and write its G q-head rows (out_row -> [G][D]).  One warp; lane i owns
+// the float4 columns i, i+32, ... of the G*D outputs.  The partials were
+// written by other warps of this grid and published before their tickets
+// (the caller has fenced after drawing the last ticket), so they are read
+// through L2 (ld.global.cg), never from a possibly stale L1 line.  A partial
+// whose running max is -inf (every token of that part skipped) adds nothing.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(merge_threads(D, G)) paged_decode_merge_kernel(const DecodeParams p) {
+__device__ __forceinline__ void merge_split_unit(const float2* ws_ml, const float* ws_o, T* out_row, int64_t a,
+                                                 int nc, int64_t NC, int W, int lane) {
   using E = Elem<T>;
-  constexpr int NT = merge_threads(D, G);
-  constexpr int ITEMS = G * D / 4;  // float4 outputs of one job
-  constexpr int NGRP = NT / ITEMS;  // contributor groups
-  extern __shared__ int mslots[];   // [W]: partial slot of each contributor, -1 if it has none
-  __shared__ float4 s_acc[NT];
-  __shared__ float2 s_ml[NT];
-
-  griddep_wait();
-  griddep_launch_dependents();
-  const int W = p.total_warps;
-  const int4 job = p.ws_jobs[blockIdx.x];
-  if (job.x < 0) return;
-  const int64_t NC = p.ws_header[0];
-  const int64_t a = job.z, b = a + job.w;
-  const int w0 = blockIdx.x;
-  const int w1 = static_cast<int>((b * W + NC - 1) / NC - 1);  // warp holding chunk b-1
-  const int nw = w1 - w0 + 1;
-  const int t = threadIdx.x;
-  for (int j = t; j < nw; j += NT) {
-    const int64_t w = w0 + j;
-    const int64_t s0 = w * NC / W, s1 = (w + 1) * NC / W;  // warps with an empty run wrote nothing
-    mslots[j] = s0 < s1 ? static_cast<int>(2 * w + (s0 >= a ? 0 : 1)) : -1;
-  }
-  __syncthreads();
-
-  const int item = t % ITEMS, grp = t / ITEMS;
-  const int g = item / (D / 4), d4 = item % (D / 4);
-  auto ml_at = [&](int slot) { return p.ws_ml[(int64_t)slot * G + g]; };
-  auto o_at = [&](int slot) { return reinterpret_cast<const float4*>(p.ws_o + ((int64_t)slot * G + g) * D)[d4]; };
-  float m = -INFINITY, l = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int j = grp;
-  for (; j + 3 * NGRP < nw; j += 4 * NGRP) {
-    int sl[4];
-    float2 ml[4];
-    float4 o[4];
+  constexpr int kItems = G * D / 4;                   // float4 outputs
+  constexpr int kPerLane = (kItems + 31) / 32;
+  constexpr int kBatch = kPerLane >= 4 ? 2 : 4;        // contributors loaded before folding
+  const int w0 = warp_of_chunk(a, NC, W);
+  const int w1 = warp_of_chunk(a + nc - 1, NC, W);
+  float m[kPerLane], l[kPerLane];
+  float4 acc[kPerLane];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      sl[u] = mslots[j + u * NGRP];
-      const int safe = sl[u] < 0 ? 0 : sl[u];  // a valid address; its values are not used
-      ml[u] = ml_at(safe);
-      o[u] = o_at(safe);
+  for (int i = 0; i < kPerLane; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+    acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int w = w0; w <= w1; w += kBatch) {
+    float2 ml[kBatch][kPerLane];
+    float4 o[kBatch][kPerLane];
+    bool use[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int wu = w + u;
+      // Warps with an empty run (more warps than chunks) wrote nothing.
+      use[u] = wu <= w1 && run_begin(wu, NC, W) < run_begin(wu + 1, NC, W);
+      const int64_t slot = use[u] ? partial_slot(wu, a, NC, W) : 0;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i) {
+        const int item = lane + 32 * i;
+        const int g = item / (D / 4), d4 = item % (D / 4);
+        if (use[u] && item < kItems) {
+          ml[u][i] = __ldcg(ws_ml + slot * G + g);
+          o[u][i] = __ldcg(reinterpret_cast<const float4*>(ws_o + (slot * G + g) * D) + d4);
+        } else {
+          ml[u][i] = make_float2(-INFINITY, 0.f);
+          o[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (sl[u] >= 0 && ml[u].x != -INFINITY) fold_partial(m, l, acc, ml[u], o[u]);
-  }
-  for (; j < nw; j += NGRP) {
-    const int slot = mslots[j];
-    if (slot < 0) continue;
-    const float2 ml = ml_at(slot);
-    if (ml.x != -INFINITY) fold_partial(m, l, acc, ml, o_at(slot));
-  }
-  if (NGRP > 1) {
-    s_acc[t] = acc;
-    s_ml[t] = make_float2(m, l);
-    __syncthreads();
-    if (grp != 0) return;
-    for (int q = 1; q < NGRP; ++q) {
-      const float2 ml = s_ml[q * ITEMS + item];
-      if (ml.x != -INFINITY) fold_partial(m, l, acc, ml, s_acc[q * ITEMS + item]);
+    for (int u = 0; u < kBatch; ++u) {
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+        if (ml[u][i].x != -INFINITY) fold_partial(m[i], l[i], acc[i], ml[u][i], o[u][i]);
     }
   }
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  T* dst = static_cast<T*>(p.out) + ((int64_t)job.x * p.num_heads + (int64_t)job.y * G + g) * D + d4 * 4;
-  uint2 u;
-  u.x = E::pack(acc.x * inv, acc.y * inv);
-  u.y = E::pack(acc.z * inv, acc.w * inv);
-  *reinterpret_cast<uint2*>(dst) = u;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int item = lane + 32 * i;
+    if (item >= kItems) continue;
+    const int g = item / (D / 4), d4 = item % (D / 4);
+    const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
+    uint2 u;
+    u.x = E::pack(acc[i].x * inv, acc[i].y * inv);
+    u.y = E::pack(acc[i].z * inv, acc[i].w * inv);
+    *reinterpret_cast<uint2*>(out_row + g * D + d4 * 4) = u;
+  }
 }
 
 }  // namespace pa

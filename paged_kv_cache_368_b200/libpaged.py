@@ -147,10 +147,12 @@ def decode_workspace_size(num_seqs: int, num_heads: int, num_kv_heads: int, head
 
 def alloc_workspace(num_seqs: int, num_heads: int, num_kv_heads: int, head_dim: int, max_context_len: int,
                     device=None) -> torch.Tensor:
+    """A decode workspace, zero-filled as pa_decode requires before its first
+    use (every call leaves it zeroed again where that matters)."""
     n = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len)
     if n == 0:
         raise LibpagedError(PA_ERR_UNSUPPORTED, "pa_decode_workspace_size")
-    return torch.empty(n, dtype=torch.uint8, device=device if device is not None else "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda")
 
 
 def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -63,10 +63,37 @@ def test_decode_host_checks(lib):
     assert _decode(lib, H=48, KVH=3) == U  # group of 16 q-heads
     assert _decode(lib, D=96) == U
     assert _decode(lib, BS=24) == U
-    assert _decode(lib, S=4096) == U
+    assert _decode(lib, S=16385) == U  # above the sequence limit
+    assert _decode(lib, KVH=1 << 15, H=1 << 15) == U
     assert _decode(lib, out=None) == I
     assert _decode(lib, q=24) == I  # misaligned
     assert _decode(lib, S=0) == libpaged.PA_OK  # nothing to do, nothing touched
+
+
+def _decode_static(lib, **kw):
+    a = dict(out=16, q=16, k=16, v=16, tables=16, mb=4, ctx=16, S=2, maxctx=64, scale=0.1, H=4, KVH=4, D=128,
+             BS=16, NB=8, dtype=0, max_ctas=0, err=None, stream=None)
+    a.update(kw)
+    return lib.pa_decode_static(a["out"], a["q"], a["k"], a["v"], a["tables"], a["mb"], a["ctx"], a["S"],
+                                a["maxctx"], a["scale"], a["H"], a["KVH"], a["D"], a["BS"], a["NB"], a["dtype"],
+                                a["max_ctas"], a["err"], a["stream"])
+
+
+def test_decode_static_host_checks(lib):
+    """The no-allocation entry point rejects bad and unsupported arguments
+    on the host, before any CUDA call (this runs without a GPU)."""
+    I, U = libpaged.PA_ERR_INVALID, libpaged.PA_ERR_UNSUPPORTED
+    assert _decode_static(lib, H=6, KVH=4) == I
+    assert _decode_static(lib, S=-1) == I
+    assert _decode_static(lib, dtype=9) == I
+    assert _decode_static(lib, max_ctas=-2) == I
+    assert _decode_static(lib, out=None) == I
+    assert _decode_static(lib, tables=18) == I  # misaligned int32
+    assert _decode_static(lib, D=80) == U
+    assert _decode_static(lib, BS=128) == U
+    assert _decode_static(lib, H=64, KVH=4) == U  # group of 16
+    assert _decode_static(lib, S=20000) == U
+    assert _decode_static(lib, S=0) == libpaged.PA_OK
 
 
 def test_reshape_host_checks(lib):
