@@ -367,7 +367,8 @@ class DecodeBench:
     def time_each_decode(self, n, flush=None):
         """Per-call ms of n pa_decode calls, an event pair around each (after
         the step's append, so the cache is the step's); with `flush` a buffer
-        larger than L2 is rewritten before every call (cold L2)."""
+        of twice the L2 is read before every call (cold L2: the lines it
+        leaves are clean, so the timed call pays no write-backs)."""
         import torch
 
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
@@ -375,7 +376,7 @@ class DecodeBench:
         for a, b in ev:
             self.lib.pa_reshape_and_cache(*self.r_args)
             if flush is not None:
-                flush.zero_()
+                flush.max()  # a read of 2x the L2
             a.record(self.stream)
             self.decode()
             b.record(self.stream)
@@ -457,7 +458,7 @@ def run_ours(args):
     lib = libpaged.load()
     dev = torch.device("cuda", local)
     peak, peak_src = measured_peak()
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.ones(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     wl = load_workload(args)
     b = DecodeBench(lib, libpaged, wl, dev)
@@ -481,7 +482,7 @@ def run_ours(args):
     # time, so that the clock samples (every 100 ms) fall inside it
     if dist is not None:
         dist.barrier()
-    n_roof = max(K, b.calls_for(1.0, elapsed_ms / K))
+    n_roof = max(K, b.calls_for(args.roofline_seconds, elapsed_ms / K))
     dec_ms = b.time_each_decode(n_roof)
     t_wall1 = time.time()
     cold_ms = b.time_each_decode(min(200, n_roof), flush=flush)
@@ -531,7 +532,7 @@ def run_ours(args):
         "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": describe(wl), "kv_bytes_per_step": kvb, "unique_kv_bytes_per_step": wl.unique_kv_bytes(),
                    "l2": (f"inputs larger than L2 ({kvb / 2**20:.0f} MiB of KV per step vs 126 MiB L2), no flush "
-                          "between timed steps; decode_us_cold_l2 flushes a 252 MiB buffer before every call"),
+                          "between timed steps; decode_us_cold_l2 reads a 252 MiB buffer before every call"),
                    "parallelism": f"{world} independent replica(s), one per GPU",
                    "step": "append (pa_reshape_and_cache) + decode with in-launch merge (pa_decode)"},
         "roofline": {"bound": "hbm", "achieved": head["decode_gbs"], "peak": peak, "unit": "GB/s",
@@ -771,6 +772,8 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (1 = LLaMA-7B-shaped layer)")
     ap.add_argument("--block-size", type=int, default=None, help="block size for workload 3 (LLaMA-13B)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--roofline-seconds", type=float, default=1.0,
+                    help="device time of the per-call roofline pass (at least K calls); 0 for profiler runs")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload table (all five workloads, LLaMA-13B at block sizes 8-64)")
     ap.add_argument("--op", choices=("step", "block_ops", "prefill"), default="step",

@@ -336,6 +336,18 @@ PA_API pa_status pa_bm_swap_sequence(pa_block_manager* from, pa_block_manager* t
  */
 PA_API pa_status pa_selftest_wait_timeout(uint64_t limit_ns, int32_t* err_flags, pa_stream_t stream);
 
+/*
+ * pa_selftest_exp2 -- evaluates, on the device, the polynomial 2^x that the
+ * multi-token kernel runs on the FMA pipe for part of its softmax
+ * exponentials, beside CUDA's exp2f on the same inputs (the pages have no
+ * counterpart): y_poly[i] = polynomial 2^x[i], y_ref[i] = exp2f(x[i]) for
+ * i < n; float32 device arrays owned by the caller.  The polynomial is
+ * specified for x < 127 with relative error below 1.0e-4, and returns 2^-125
+ * for x <= -125 (including -inf).  Asynchronous on `stream`; PA_ERR_INVALID
+ * for n < 0 or a NULL array.
+ */
+PA_API pa_status pa_selftest_exp2(const float* x, float* y_poly, float* y_ref, int64_t n, pa_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 PA_API const char* pa_status_string(pa_status status);
 

@@ -10,22 +10,29 @@ namespace pa {
 
 constexpr int kMaxDevices = 64;
 
-// Decode workspace for a grid of W warps and group size G, head_dim D:
-//   tickets [W] int32   per split unit (indexed by the warp holding its first
-//                       chunk): chunks accounted for so far; zero between calls
-//   ml      [2W][G]     float2 (running max in log2 units, running sum)
-//   o       [2W][G][D]  float  un-normalised partial outputs
+// Decode workspace for a grid of W warps on a device whose largest grid has
+// Wmax warps (SM count x kMaxWarpsPerCta), group size G, head_dim D:
+//   tickets [Wmax] int32  per split unit (indexed by the warp holding its
+//                         first chunk): chunks accounted for so far; zero
+//                         between calls
+//   ml      [2W][G]       float2 (running max in log2 units, running sum)
+//   o       [2W][G][D]    float  un-normalised partial outputs
 // Two partial slots per warp: a warp's run has at most two segments that
-// cover only part of a unit (its first and its last).
+// cover only part of a unit (its first and its last).  The ticket region has
+// the same size for every call on a device, so the partials of one call
+// never land on the counters of another that reuses the workspace with a
+// larger grid.
+constexpr int kMaxWarpsPerCta = 8;
+
 struct WsLayout {
   size_t tickets, ml, o, total;
 };
 
 constexpr size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-constexpr WsLayout ws_layout(int W, int G, int D) {
-  return WsLayout{0, round256(size_t(W) * 4), round256(size_t(W) * 4) + round256(size_t(2) * W * G * 8),
-                  round256(size_t(W) * 4) + round256(size_t(2) * W * G * 8) + size_t(2) * W * G * D * 4};
+constexpr WsLayout ws_layout(int W, int Wmax, int G, int D) {
+  return WsLayout{0, round256(size_t(Wmax) * 4), round256(size_t(Wmax) * 4) + round256(size_t(2) * W * G * 8),
+                  round256(size_t(Wmax) * 4) + round256(size_t(2) * W * G * 8) + size_t(2) * W * G * D * 4};
 }
 
 struct DecodePlan {

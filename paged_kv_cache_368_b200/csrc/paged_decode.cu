@@ -25,7 +25,9 @@
 //    log-sum-exp and writes the output, in the same launch: no warp waits
 //    for another and there is no second kernel.
 //  * Each warp is its own producer: lane 0 issues TMA tile loads (128-byte
-//    swizzle, L2 evict-first) of the K and V rows of chunk k+DEPTH into a
+//    swizzle; L2 evict-first, except each unit's first 1024 tokens, where
+//    shared prefix blocks live, at the normal policy) of the K and V rows of
+//    chunk k+DEPTH into a
 //    per-warp ring of shared-memory stages, completion counted on an
 //    mbarrier, while the warp computes on chunk k.  Block-table entries for
 //    the next 32 chunks are fetched with one coalesced load (one per lane)
@@ -189,7 +191,7 @@ pa_status plan_decode(int num_seqs, int max_blocks_per_seq, int max_context_len,
   plan->ctx_cap = static_cast<int>(cap64);
   plan->warps = warps_for(head_dim, G);
   plan->ctas = 0;
-  plan->layout = ws_layout(0, G, head_dim);
+  plan->layout = ws_layout(0, 0, G, head_dim);
   plan->upper_chunks = upper;
   return PA_OK;
 }
@@ -208,7 +210,7 @@ pa_status plan_decode_grid(int max_ctas, DecodePlan* plan) {
                                                                             (plan->warps * 4))));
   if (max_ctas > 0) ctas = std::min(ctas, max_ctas);
   plan->ctas = ctas;
-  plan->layout = ws_layout(ctas * plan->warps, plan->G, plan->head_dim);
+  plan->layout = ws_layout(ctas * plan->warps, sms * kMaxWarpsPerCta, plan->G, plan->head_dim);
   return PA_OK;
 }
 
@@ -226,7 +228,7 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_
   const int sms = pa::device_sms(dev);
   if (sms <= 0) return 0;
   // The largest grid this shape can launch on this device (one CTA per SM).
-  return pa::ws_layout(sms * pa::warps_for(head_dim, G), G, head_dim).total;
+  return pa::ws_layout(sms * pa::warps_for(head_dim, G), sms * pa::kMaxWarpsPerCta, G, head_dim).total;
 }
 
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -33,6 +33,7 @@ __host__ __device__ constexpr bool uses_mma(int G) { return G >= 4; }
 __host__ __device__ constexpr int warps_for(int D, int G) {
   return D == 64 ? 8 : (uses_mma(G) ? PA_MMA_WARPS : PA_CORE_WARPS);
 }
+static_assert(PA_CORE_WARPS <= 8 && PA_MMA_WARPS <= 8, "the workspace's ticket region holds 8 warps per SM");
 __host__ __device__ constexpr int depth_for(int D, int G) {
   return D == 64 ? PA_D64_DEPTH : (uses_mma(G) ? PA_MMA_DEPTH : PA_CORE_DEPTH);
 }
@@ -138,9 +139,23 @@ __device__ __forceinline__ ChunkRaw chunk_load(const DecodeParams& p, const int*
 //   sh    = seq | kv_head << 16
 //   flags = valid tokens (bits 0-4) | first row in the block (bits 5-10)
 //           | first chunk of its unit (bit 11) | last chunk of its unit (bit 12)
+//           | one of the unit's first kHeadChunks chunks (bit 13)
 //   p0/p1 = physical block(s); p1 = -1 when the chunk has one block.
 constexpr int kFlagStart = 1 << 11;
 constexpr int kFlagEnd = 1 << 12;
+constexpr int kFlagHead = 1 << 13;
+
+// L2 residency: blocks shared between sequences (a common prompt prefix,
+// beams forked from one request: "【infra之路】10-PagedAttention 与 KV Cache
+// 管理", section 4.3) sit at the front of their sequences.  The first
+// kHeadChunks chunks (1024 tokens) of every unit are loaded with the normal
+// L2 policy and everything after them evict-first, so a shared front block
+// read by one sequence is still in L2 when its sharers read it, while the
+// once-read rest streams through without displacing it.
+#ifndef PA_HEAD_CHUNKS
+#define PA_HEAD_CHUNKS 64
+#endif
+constexpr int kHeadChunks = PA_HEAD_CHUNKS;
 
 struct ChunkInfo {
   int sh, flags, p0, p1, c, nc;
@@ -165,7 +180,8 @@ __device__ __forceinline__ ChunkInfo chunk_finalize(const DecodeParams& p, const
   }
   const int row0 = p.block_size >= kChunk ? t0 % p.block_size : 0;
   ci.sh = r.seq | (r.head << 16);
-  ci.flags = valid | (row0 << 5) | (r.c == 0 ? kFlagStart : 0) | (r.c == r.nc - 1 ? kFlagEnd : 0);
+  ci.flags = valid | (row0 << 5) | (r.c == 0 ? kFlagStart : 0) | (r.c == r.nc - 1 ? kFlagEnd : 0) |
+             (r.c < kHeadChunks ? kFlagHead : 0);
   ci.p0 = r.p0;
   ci.p1 = p1;
   return ci;
@@ -570,7 +586,8 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     }
   }
 
-  const uint64_t policy = l2_evict_first_policy();
+  const uint64_t policy_stream = l2_evict_first_policy();
+  const uint64_t policy_head = l2_evict_normal_policy();
   const int rows_per_block = p.block_size < kChunk ? p.block_size : kChunk;
   const uint32_t box_bytes = rows_per_block * 128;
   const T* qbase = static_cast<const T*>(p.q);
@@ -592,6 +609,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     const int row0 = (flags >> 5) & 63;
     const int head = sh >> 16, seq = sh & 0xffff;
     const int nblk = valid > 0 ? (p1 >= 0 ? 2 : 1) : 0;
+    const uint64_t policy = (flags & kFlagHead) ? policy_head : policy_stream;
     const uint32_t bytes = nblk * (D / 64) * box_bytes * 2 + (seg_start ? SH::kQBytes : 0);
     mbar_arrive_expect_tx(bar, bytes);
     const uint32_t kt = tiles + stage * SH::kStageBytes;

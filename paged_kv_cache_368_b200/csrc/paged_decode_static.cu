@@ -54,7 +54,7 @@ constexpr size_t largest_need(int sms) {
   size_t need = 0;
   for (int D : {64, 128})
     for (int G : {1, 2, 4, 8}) {
-      const size_t n = pa::ws_layout(sms * pa::warps_for(D, G), G, D).total;
+      const size_t n = pa::ws_layout(sms * pa::warps_for(D, G), sms * pa::kMaxWarpsPerCta, G, D).total;
       need = n > need ? n : need;
     }
   return need;
@@ -62,8 +62,9 @@ constexpr size_t largest_need(int sms) {
 static_assert(largest_need(kLargestGridSMs) <= kStaticScratchBytes,
               "the static scratch must hold the workspace of every supported shape on a 148-SM GPU");
 
-// Ticket counters of the largest grid any shape can launch on `sms` SMs.
-size_t ticket_bytes(int sms) { return pa::ws_layout(sms * 8, 1, 64).ml; }
+// The ticket counters at the front of the scratch (the same region for every
+// call on a device with `sms` SMs).
+size_t ticket_bytes(int sms) { return pa::ws_layout(0, sms * pa::kMaxWarpsPerCta, 1, 64).ml; }
 
 }  // namespace
 

@@ -1,7 +1,13 @@
-// Self-test of the bounded barrier wait every kernel of the library relies on
-// (no counterpart on the pages): one CTA waits on shared-memory barriers that
-// nothing ever completes and must give up after the given limit, flag the
-// timeout and return, leaving the context usable.
+// Device self-tests (no counterpart on the pages):
+//  * the bounded barrier wait every kernel of the library relies on: one CTA
+//    waits on shared-memory barriers that nothing ever completes and must give
+//    up after the given limit, flag the timeout and return, leaving the
+//    context usable;
+//  * the polynomial 2^x of the multi-token kernel (exp2_poly.cuh), evaluated
+//    beside CUDA's exp2f on the same inputs.
+#include <algorithm>
+
+#include "exp2_poly.cuh"
 #include "pa_host.h"
 #include "tcgen05.cuh"
 
@@ -27,8 +33,25 @@ __global__ void __launch_bounds__(32, 1) wait_timeout_kernel(uint64_t limit_ns, 
   }
 }
 
+__global__ void exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    y_poly[i] = exp2_poly(v);
+    y_ref[i] = exp2f(v);
+  }
+}
+
 }  // namespace
 }  // namespace pa
+
+extern "C" pa_status pa_selftest_exp2(const float* x, float* y_poly, float* y_ref, int64_t n, pa_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_ref))) return PA_ERR_INVALID;
+  if (n == 0) return PA_OK;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096));
+  pa::exp2_selftest_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y_poly, y_ref, n);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : pa::fail(PA_ERR_CUDA, "launching exp2_selftest_kernel", e);
+}
 
 extern "C" pa_status pa_selftest_wait_timeout(uint64_t limit_ns, int32_t* err_flags, pa_stream_t stream) {
   if (!err_flags || limit_ns == 0 || limit_ns > 100000000ull) return PA_ERR_INVALID;

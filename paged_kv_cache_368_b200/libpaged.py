@@ -28,7 +28,7 @@ SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_
            "pa_decode_step_host", "pa_step_inputs_layout", "pa_prefill", "pa_prefill_mma", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
            "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slot",
            "pa_bm_free_sequence", "pa_bm_context_len", "pa_bm_block_table", "pa_bm_blocks_needed_to_append",
-           "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_selftest_wait_timeout", "pa_status_string",
+           "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_selftest_wait_timeout", "pa_selftest_exp2", "pa_status_string",
            "pa_version", "pa_last_error")
 
 _lib: Optional[ctypes.CDLL] = None
@@ -77,6 +77,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, f).restype = _i32
     lib.pa_selftest_wait_timeout.argtypes = [_c.c_uint64, _vp, _vp]
     lib.pa_selftest_wait_timeout.restype = _i32
+    lib.pa_selftest_exp2.argtypes = [_vp, _vp, _vp, _i64, _vp]
+    lib.pa_selftest_exp2.restype = _i32
     lib.pa_status_string.argtypes = [_i32]
     lib.pa_status_string.restype = _c.c_char_p
     lib.pa_version.argtypes = []
@@ -315,6 +317,18 @@ def selftest_wait_timeout(err_flags: torch.Tensor, limit_ns: int = 2_000_000, st
     st = load().pa_selftest_wait_timeout(int(limit_ns), _dev_ptr(err_flags, "err_flags"), _stream(stream))
     if st != PA_OK:
         raise LibpagedError(st, "pa_selftest_wait_timeout")
+
+
+def selftest_exp2(x: torch.Tensor, stream=None):
+    """(polynomial 2^x, exp2f(x)) evaluated on the device for a float32 CUDA tensor."""
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    y_poly, y_ref = torch.empty_like(x), torch.empty_like(x)
+    st = load().pa_selftest_exp2(_dev_ptr(x, "x"), _dev_ptr(y_poly, "y_poly"), _dev_ptr(y_ref, "y_ref"), x.numel(),
+                                 _stream(stream))
+    if st != PA_OK:
+        raise LibpagedError(st, "pa_selftest_exp2")
+    return y_poly, y_ref
 
 
 def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_pairs: torch.Tensor,

@@ -150,6 +150,9 @@ def test_prefill_host_checks(lib, entry):
 
 def test_selftest_host_checks(lib):
     I = libpaged.PA_ERR_INVALID
+    assert lib.pa_selftest_exp2(None, None, None, 5, None) == I
+    assert lib.pa_selftest_exp2(16, 16, 16, -1, None) == I
+    assert lib.pa_selftest_exp2(None, None, None, 0, None) == libpaged.PA_OK
     assert lib.pa_selftest_wait_timeout(1000, None, None) == I  # no flag words
     assert lib.pa_selftest_wait_timeout(0, 16, None) == I  # zero limit
     assert lib.pa_selftest_wait_timeout(200_000_000, 16, None) == I  # above 0.1 s

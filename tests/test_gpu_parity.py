@@ -317,22 +317,23 @@ def test_decode_step_from_host_buffers():
 
 
 def test_merge_tickets_return_to_zero_and_workspace_reuse_is_exact():
-    """The in-launch merge counts each split unit's chunks on a ticket counter
-    in the workspace and leaves every counter at zero: one zeroed workspace
-    reused across shapes and grid caps gives the same bits as a fresh one."""
-    shared = None
+    """The in-launch merge counts each split unit's chunks on ticket counters
+    at the front of the workspace (one int32 per warp of the largest grid:
+    SMs x 8, the same region for every call) and leaves every counter at
+    zero: one zeroed workspace reused across shapes and grid caps (a capped
+    grid's partials must not land on a larger grid's counters) gives the same
+    bits as a fresh one, and every output row is written by every call."""
+    shared = torch.zeros(64 << 20, dtype=torch.uint8, device="cuda")
+    nbytes = 4 * 8 * torch.cuda.get_device_properties(0).multi_processor_count
     for seed, g, max_ctas in ((201, 4, 0), (202, 1, 3), (203, 8, 7), (204, 2, 0), (201, 4, 2)):
         wl = inputs.random_case(seed, num_seqs=7, num_heads=2 * g, num_kv_heads=2, head_dim=128, block_size=16,
                                 dtype="bf16", ctx_lo=1, ctx_hi=5000)
-        fresh = DeviceState(wl, full_pool=True)
-        want = fresh.step(max_ctas=max_ctas)
-        if shared is None:
-            shared = torch.zeros(64 << 20, dtype=torch.uint8, device="cuda")
+        want = DeviceState(wl, full_pool=True).step(max_ctas=max_ctas)
         ds = DeviceState(wl, full_pool=True)
         ds.ws = shared
         for _ in range(2):
-            got = ds.step(max_ctas=max_ctas)
-            assert np.array_equal(got, want), (seed, max_ctas)  # the repeated append rewrites the same rows
-        sms = torch.cuda.get_device_properties(0).multi_processor_count
-        assert int(shared[: sms * 6 * 4].count_nonzero().item()) == 0
+            ds.out.fill_(float("nan"))  # a row the call fails to write stays NaN
+            got = ds.step(max_ctas=max_ctas)  # the repeated append rewrites the same rows
+            assert np.array_equal(got, want), (seed, max_ctas)
+            assert int(shared[:nbytes].count_nonzero().item()) == 0, (seed, max_ctas)
         assert int(ds.err.item()) == 0

@@ -127,3 +127,21 @@ def test_malformed_offsets_touch_nothing():
     ref = oracle.prefill(q[:20], cu[:2], k, v, wl.block_tables[:1], wl.context_lens[:1], wl.scale, "bf16")
     assert_close(out[:20], ref, "bf16", "first sequence")
     assert np.all(out[20:] == to_raw(torch.full((1,), float("nan"), dtype=torch.bfloat16))[0])  # untouched
+
+
+def test_polynomial_exp2_against_exp2f():
+    """The softmax's FMA-pipe 2^x, on the device, against CUDA's exp2f on the
+    same inputs: relative error below 1.0e-4 over the range the kernel feeds it
+    (scaled scores minus the reference max, up to the 2^8 head room), and the
+    clamp to 2^-125 below."""
+    x = torch.cat([torch.linspace(-124.9, 8.5, 1 << 20), torch.arange(-124, 9, dtype=torch.float32),
+                   torch.rand(1 << 18) - 0.5]).cuda()
+    y_poly, y_ref = libpaged.selftest_exp2(x)
+    torch.cuda.synchronize()
+    rel = ((y_poly.double() - y_ref.double()) / y_ref.double()).abs()
+    assert float(rel.max()) < 1.0e-4
+    exact = torch.exp2(x.double())
+    assert float(((y_ref.double() - exact) / exact).abs().max()) < 1e-6  # exp2f itself: the yardstick
+    low, _ = libpaged.selftest_exp2(torch.tensor([float("-inf"), -1e30, -300.0, -125.0], device="cuda"))
+    torch.cuda.synchronize()
+    assert float(((low.double() / 2.0**-125) - 1).abs().max()) < 1.0e-4
