@@ -340,8 +340,9 @@ PA_API pa_status pa_selftest_wait_timeout(uint64_t limit_ns, int32_t* err_flags,
  * pa_selftest_exp2 -- evaluates, on the device, the polynomial 2^x that the
  * multi-token kernel runs on the FMA pipe for part of its softmax
  * exponentials, beside CUDA's exp2f on the same inputs (the pages have no
- * counterpart): y_poly[i] = polynomial 2^x[i], y_ref[i] = exp2f(x[i]) for
- * i < n; float32 device arrays owned by the caller.  The polynomial is
+ * counterpart): y_poly[i] = polynomial 2^x[i] (the scalar form for even i,
+ * the packed two-input form for odd i), y_ref[i] = exp2f(x[i]) for i < n;
+ * float32 device arrays owned by the caller.  The polynomial is
  * specified for x < 127 with relative error below 1.0e-4, and returns 2^-125
  * for x <= -125 (including -inf).  Asynchronous on `stream`; PA_ERR_INVALID
  * for n < 0 or a NULL array.

@@ -25,9 +25,7 @@
 //    log-sum-exp and writes the output, in the same launch: no warp waits
 //    for another and there is no second kernel.
 //  * Each warp is its own producer: lane 0 issues TMA tile loads (128-byte
-//    swizzle; L2 evict-first, except each unit's first 1024 tokens, where
-//    shared prefix blocks live, at the normal policy) of the K and V rows of
-//    chunk k+DEPTH into a
+//    swizzle, L2 evict-first) of the K and V rows of chunk k+DEPTH into a
 //    per-warp ring of shared-memory stages, completion counted on an
 //    mbarrier, while the warp computes on chunk k.  Block-table entries for
 //    the next 32 chunks are fetched with one coalesced load (one per lane)

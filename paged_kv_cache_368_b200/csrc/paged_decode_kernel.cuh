@@ -147,13 +147,14 @@ constexpr int kFlagHead = 1 << 13;
 
 // L2 residency: blocks shared between sequences (a common prompt prefix,
 // beams forked from one request: "【infra之路】10-PagedAttention 与 KV Cache
-// 管理", section 4.3) sit at the front of their sequences.  The first
-// kHeadChunks chunks (1024 tokens) of every unit are loaded with the normal
-// L2 policy and everything after them evict-first, so a shared front block
-// read by one sequence is still in L2 when its sharers read it, while the
-// once-read rest streams through without displacing it.
+// 管理", section 4.3) sit at the front of their sequences.  With
+// PA_HEAD_CHUNKS > 0 the first PA_HEAD_CHUNKS chunks of every unit are loaded
+// with the normal L2 policy and everything after them evict-first, so that a
+// shared front block read by one sequence can still be in L2 when its
+// sharers read it.  Off by default: at 64 chunks (1024 tokens) it cost ~2 us
+// per call on the LLaMA-7B workload, where nothing is shared.
 #ifndef PA_HEAD_CHUNKS
-#define PA_HEAD_CHUNKS 64
+#define PA_HEAD_CHUNKS 0
 #endif
 constexpr int kHeadChunks = PA_HEAD_CHUNKS;
 
@@ -569,11 +570,42 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
   const int64_t c0 = run_begin(gw, NC, W), c1 = run_begin(gw + 1, NC, W);
   const int n = static_cast<int>(c1 - c0);
 
+  // The run's split parts.  Its first segment (containing the run's first
+  // chunk) and its last segment (containing the last chunk) may each cover
+  // only part of a unit; every other segment is a whole unit.
+  UnitPos uf{0, 0, 0, 1}, ul{0, 0, 0, 1};
+  int64_t af = 0, al = 0;  // global first chunks of those two units
+  bool part_f = false, part_l = false;
+  int mine_f = 0, mine_l = 0;  // chunks of those units in this run
+  if (n > 0) {
+    uf = unit_pos(p, prefix, c0);
+    ul = unit_pos(p, prefix, c1 - 1);
+    af = c0 - uf.c;
+    al = c1 - 1 - ul.c;
+    if (af == al) {  // the whole run lies in one unit
+      part_f = !(uf.c == 0 && ul.c == ul.nc - 1);
+      mine_f = n;
+    } else {
+      part_f = uf.c != 0;
+      mine_f = uf.nc - uf.c;
+      part_l = ul.c != ul.nc - 1;
+      mine_l = ul.c + 1;
+    }
+  }
+  // Processing order: the last segment first, when it is a split part, then
+  // the run from its start, which begins with the first segment.  Both split
+  // parts are thus done early and their merges (below) overlap the other
+  // warps' streaming instead of lengthening the kernel's tail.  Virtual index
+  // k in [0, n) is physical chunk c0 + phys(k).
+  const int shift = part_l ? n - mine_l : 0;
+  auto phys = [&](int k) { return k + shift < n ? k + shift : k + shift - n; };
+  auto gchunk = [&](int k) { return k < n ? c0 + phys(k) : c1; };  // c1: past the run
+
   // Chunk windows: `cur` holds chunks [kb, kb+32), `nxt` [kb+32, kb+64), and
-  // the raw loads of [kb+64, kb+96) are in flight.
-  const ChunkRaw r0 = chunk_load(p, prefix, c0 + lane, c1);
-  const ChunkRaw r1 = chunk_load(p, prefix, c0 + 32 + lane, c1);
-  ChunkRaw rnext = chunk_load(p, prefix, c0 + 64 + lane, c1);
+  // the raw loads of [kb+64, kb+96) are in flight (processing order).
+  const ChunkRaw r0 = chunk_load(p, prefix, gchunk(lane), c1);
+  const ChunkRaw r1 = chunk_load(p, prefix, gchunk(32 + lane), c1);
+  ChunkRaw rnext = chunk_load(p, prefix, gchunk(64 + lane), c1);
   ChunkInfo cur = chunk_finalize(p, r0);
   ChunkInfo nxt = chunk_finalize(p, r1);
   int kb = 0;
@@ -591,6 +623,10 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
   const int rows_per_block = p.block_size < kChunk ? p.block_size : kChunk;
   const uint32_t box_bytes = rows_per_block * 128;
   const T* qbase = static_cast<const T*>(p.q);
+  // A segment starts at the first chunk processed, at a unit's first chunk,
+  // and where the processing order wraps to the run's first chunk.
+  auto seg_starts = [&](int k, int flags) { return k == 0 || (flags & kFlagStart) || phys(k) == 0; };
+  auto seg_ends = [&](int k, int flags) { return k == n - 1 || (flags & kFlagEnd) || phys(k) == n - 1; };
 
   // Issue the loads of chunk k into its stage (lane 0; all lanes shuffle).
   auto issue = [&](int k) {
@@ -604,7 +640,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     if (lane != 0) return;
     const int stage = warp * DEPTH + (k % DEPTH);
     uint64_t* bar = &bars[stage];
-    const bool seg_start = (k == 0) || (flags & kFlagStart);
+    const bool seg_start = seg_starts(k, flags);
     const int valid = flags & 31;
     const int row0 = (flags >> 5) & 63;
     const int head = sh >> 16, seq = sh & 0xffff;
@@ -615,12 +651,12 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     const uint32_t kt = tiles + stage * SH::kStageBytes;
     const uint32_t vt = kt + SH::kTileBytes;
     for (int b = 0; b < nblk; ++b) {
-      const int phys = b == 0 ? p0 : p1;
+      const int phys_blk = b == 0 ? p0 : p1;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const uint32_t off = c * 2048 + b * 1024;
-        tma_load_4d(kt + off, &kmap, bar, 64 * c, row0, head, phys, policy);
-        tma_load_4d(vt + off, &vmap, bar, 64 * c, row0, head, phys, policy);
+        tma_load_4d(kt + off, &kmap, bar, 64 * c, row0, head, phys_blk, policy);
+        tma_load_4d(vt + off, &vmap, bar, 64 * c, row0, head, phys_blk, policy);
       }
     }
     if (seg_start) {
@@ -629,12 +665,39 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     }
   };
 
+  // Split units: for each split part the warp adds its chunk count to the
+  // unit's ticket counter, right after writing the part's partial; the warp
+  // whose addition completes the unit's count merges every part and writes
+  // the output, so no warp ever waits for another.
+  bool ticket_f = false, ticket_l = false;
+  auto take_ticket = [&](bool first) {
+    const int64_t a = first ? af : al;
+    const UnitPos& u = first ? uf : ul;
+    const int mine = first ? mine_f : mine_l;
+    __threadfence();  // this lane's partial stores before the ticket
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      int* t = p.ws_tickets + warp_of_chunk(a, NC, W);
+      const int before = atomicAdd(t, mine);
+      last = before + mine == u.nc;
+      if (last) *t = 0;  // all parts counted; nobody else touches it in this launch
+    }
+    if (__shfl_sync(kFull, last, 0)) {
+      __threadfence();  // the other parts' stores, published before their tickets
+      merge_split_unit<T, D, G>(p.ws_ml, p.ws_o,
+                                static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D, a,
+                                u.nc, NC, W, lane);
+    }
+    (first ? ticket_f : ticket_l) = true;
+  };
+
   for (int i = 0; i < DEPTH && i < n; ++i) issue(i);
 
   Warp st;
   st.reset();
   bool seg_from_unit_start = false;
-  bool first_seg = true;
+  bool seg_has_run_start = false;  // the segment holds the run's first chunk: partial slot 0, else 1
   bool timed_out = false;
   int k = 0;
   for (; k < n; ++k) {
@@ -642,7 +705,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
       cur = nxt;
       nxt = chunk_finalize(p, rnext);
       kb += 32;
-      rnext = chunk_load(p, prefix, c0 + kb + 64 + lane, c1);
+      rnext = chunk_load(p, prefix, gchunk(kb + 64 + lane), c1);
     }
     const int d = k - kb;
     const int flags = __shfl_sync(kFull, cur.flags, d);
@@ -656,12 +719,13 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
       timed_out = true;
       break;
     }
-    const bool seg_start = (k == 0) || (flags & kFlagStart);
-    const bool seg_end = (k == n - 1) || (flags & kFlagEnd);
+    const bool seg_start = seg_starts(k, flags);
+    const bool seg_end = seg_ends(k, flags);
     if (seg_start) {
       st.reset();
       st.load_q(qslots + stage * SH::kQBytes, p.scale_log2, lane);
       seg_from_unit_start = (flags & kFlagStart) != 0;
+      seg_has_run_start = phys(k) == 0;
     }
     const int valid = flags & 31;
     const uint32_t kt = tiles + stage * SH::kStageBytes;
@@ -686,10 +750,10 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
       if (seg_from_unit_start && unit_end) {
         st.write_out(static_cast<T*>(p.out) + ((int64_t)seq * H + (int64_t)kvh * G) * D, lane);
       } else {
-        const int slot = 2 * gw + (first_seg ? 0 : 1);
+        const int slot = 2 * gw + (seg_has_run_start ? 0 : 1);
         st.write_partial(p.ws_o + (int64_t)slot * G * D, p.ws_ml + (int64_t)slot * G, lane);
+        take_ticket(seg_has_run_start);
       }
-      first_seg = false;
     }
   }
   if (timed_out) {
@@ -697,40 +761,10 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     // Let this warp's copies in flight land before the CTA can exit.
     for (int kk = k; kk < n && kk < k + DEPTH; ++kk)
       mbar_wait_bounded(&bars[warp * DEPTH + (kk % DEPTH)], (kk / DEPTH) & 1, kWaitLimitNs);
-  }
-  if (n == 0) return;
-
-  // Split units: the run's first and last segments may each cover only part
-  // of a unit.  For each such part the warp adds its chunk count to the
-  // unit's ticket counter; the warp whose addition completes the unit's
-  // count merges every part and writes the output, so no warp ever waits
-  // for another.  Tickets are taken after the run (also when a wait gave
-  // up, so the counters always return to zero; the outputs are then flagged
-  // as not written).
-  const UnitPos uf = unit_pos(p, prefix, c0), ul = unit_pos(p, prefix, c1 - 1);
-  const int64_t af = c0 - uf.c, al = c1 - 1 - ul.c;  // global first chunks of the two units
-  auto take_ticket = [&](int64_t a, const UnitPos& u, int mine) {
-    __threadfence();  // this lane's partial stores before the ticket
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      int* t = p.ws_tickets + warp_of_chunk(a, NC, W);
-      const int before = atomicAdd(t, mine);
-      last = before + mine == u.nc;
-      if (last) *t = 0;  // all parts counted; nobody else touches it in this launch
-    }
-    if (__shfl_sync(kFull, last, 0)) {
-      __threadfence();  // the other parts' stores, published before their tickets
-      merge_split_unit<T, D, G>(p.ws_ml, p.ws_o,
-                                static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D, a,
-                                u.nc, NC, W, lane);
-    }
-  };
-  if (af == al) {  // the whole run lies in one unit
-    if (!(uf.c == 0 && ul.c == ul.nc - 1)) take_ticket(af, uf, n);
-  } else {
-    if (uf.c != 0) take_ticket(af, uf, uf.nc - uf.c);
-    if (ul.c != ul.nc - 1) take_ticket(al, ul, ul.c + 1);
+    // The split parts not reached still count their chunks, so the counters
+    // return to zero (their outputs are flagged as not written).
+    if (part_f && !ticket_f) take_ticket(true);
+    if (part_l && !ticket_l) take_ticket(false);
   }
 }
 

@@ -54,7 +54,10 @@ __device__ __forceinline__ void merge_split_unit(const float2* ws_ml, const floa
   using E = Elem<T>;
   constexpr int kItems = G * D / 4;                   // float4 outputs
   constexpr int kPerLane = (kItems + 31) / 32;
-  constexpr int kBatch = kPerLane >= 4 ? 2 : 4;        // contributors loaded before folding
+  // contributors loaded before folding: about eight float4 columns in flight
+  // per lane, whatever G (the merge runs inside the streaming loop and its
+  // registers add to the loop's)
+  constexpr int kBatch = kPerLane >= 8 ? 1 : 8 / kPerLane;
   const int w0 = warp_of_chunk(a, NC, W);
   const int w1 = warp_of_chunk(a + nc - 1, NC, W);
   float m[kPerLane], l[kPerLane];

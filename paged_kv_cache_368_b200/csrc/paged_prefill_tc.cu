@@ -280,7 +280,9 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     constexpr uint32_t id_pv = tc5::f16_idesc(fmt, BM, D, 0, 1);
     const uint32_t leader = tc5::elect_one();
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-      const bool got = tc5::wait(bar, parity, kWaitNs);
+      // one plain probe first: most of these waits are already satisfied,
+      // and the suspending form costs the pacing warp ~100 cycles even then
+      const bool got = tc5::wait_fast(bar, parity, kWaitNs);
       return __all_sync(kFull, got);
     };
     int kv_seen = -1;  // highest tile whose copies this warp has already waited for
@@ -421,18 +423,19 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;
       // P row, 16-bit, two keys per tensor-memory column, into the front of
       // this tile's S buffer (already read).
+      // Scale-and-shift and the row sum run as packed fp32x2 operations (one
+      // instruction for two keys); the exponentials on the special-function unit.
       uint32_t pk[BN / 2];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float ls[4][2] = {};
 #pragma unroll
-      for (int c8 = 0; c8 < BN / 8; ++c8) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(fmaf(sv[c8 * 8 + e], p.scale_log2, -mref));
-        ls[c8 & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]) + ((pv[4] + pv[5]) + (pv[6] + pv[7]));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pk[c8 * 4 + e] = E::pack(pv[2 * e], pv[2 * e + 1]);
+      for (int i = 0; i < BN / 2; ++i) {
+        float x0, x1;
+        tc5::fma2(x0, x1, sv[2 * i], sv[2 * i + 1], p.scale_log2, -mref);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        tc5::add2(ls[i & 3][0], ls[i & 3][1], p0, p1);
+        pk[i] = E::pack(p0, p1);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += ((ls[0][0] + ls[0][1]) + (ls[1][0] + ls[1][1])) + ((ls[2][0] + ls[2][1]) + (ls[3][0] + ls[3][1]));
       tc5::st32(sj, pk);
       // V rows at keys >= the CTA's last visible key carry zero weight for
       // every row but may hold no data: the last group with rows zeroes them

@@ -33,10 +33,18 @@ __global__ void __launch_bounds__(32, 1) wait_timeout_kernel(uint64_t limit_ns, 
   }
 }
 
+// y_poly: the scalar polynomial for even i, the packed two-input form (on
+// the pair x[i-1], x[i]) for odd i, so both forms the kernels use are checked.
 __global__ void exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int64_t n) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const float v = x[i];
-    y_poly[i] = exp2_poly(v);
+    if (i & 1) {
+      float a, b;
+      exp2_poly2(a, b, x[i - 1], v);
+      y_poly[i] = b;
+    } else {
+      y_poly[i] = exp2_poly(v);
+    }
     y_ref[i] = exp2f(v);
   }
 }
