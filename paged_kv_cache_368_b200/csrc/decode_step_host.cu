@@ -8,6 +8,11 @@
 // per-step tensors cross PCIe.  They travel packed in one staging buffer
 // (layout from pa_step_inputs_layout), so a step costs one host-to-device
 // and one device-to-host copy.
+//
+// pa_decode_step_host_pipelined is the same step for a serving loop: its
+// host-to-device copy runs on a second stream, into one of two staging
+// buffers used in turn, so that it overlaps the previous step's kernels
+// instead of preceding them.
 #include "pa_device.cuh"
 
 namespace {
@@ -35,6 +40,30 @@ extern "C" size_t pa_step_inputs_layout(int num_seqs, int num_heads, int num_kv_
   return off;
 }
 
+namespace {
+
+// Append and decode from a staging buffer already on the device (both on `stream`).
+pa_status step_kernels(void* d_inputs, const size_t off[6], void* d_out, void* k_cache, void* v_cache, int num_seqs,
+                       int max_blocks_per_seq, int max_context_len, float scale, int num_heads, int num_kv_heads,
+                       int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype, void* workspace,
+                       size_t workspace_bytes, int32_t* err_flags, pa_stream_t stream) {
+  uint8_t* d = static_cast<uint8_t*>(d_inputs);
+  const void* d_q = d + off[0];
+  const void* d_key = d + off[1];
+  const void* d_value = d + off[2];
+  const int64_t* d_slots = reinterpret_cast<const int64_t*>(d + off[3]);
+  const int32_t* d_tables = reinterpret_cast<const int32_t*>(d + off[4]);
+  const int32_t* d_ctx = reinterpret_cast<const int32_t*>(d + off[5]);
+  pa_status st = pa_reshape_and_cache(d_key, d_value, k_cache, v_cache, d_slots, num_seqs, num_kv_heads, head_dim,
+                                      block_size, num_blocks, dtype, err_flags, stream);
+  if (st != PA_OK) return st;
+  return pa_decode(d_out, d_q, k_cache, v_cache, d_tables, max_blocks_per_seq, d_ctx, num_seqs, max_context_len,
+                   scale, num_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype, workspace,
+                   workspace_bytes, 0, err_flags, stream);
+}
+
+}  // namespace
+
 extern "C" pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, void* h_out, void* d_out,
                                          void* k_cache, void* v_cache, int num_seqs, int max_blocks_per_seq,
                                          int max_context_len, float scale, int num_heads, int num_kv_heads,
@@ -50,22 +79,50 @@ extern "C" pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, v
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(d_inputs, h_inputs, total, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host: host-to-device copy", e);
-  uint8_t* d = static_cast<uint8_t*>(d_inputs);
-  const void* d_q = d + off[0];
-  const void* d_key = d + off[1];
-  const void* d_value = d + off[2];
-  const int64_t* d_slots = reinterpret_cast<const int64_t*>(d + off[3]);
-  const int32_t* d_tables = reinterpret_cast<const int32_t*>(d + off[4]);
-  const int32_t* d_ctx = reinterpret_cast<const int32_t*>(d + off[5]);
-  pa_status st = pa_reshape_and_cache(d_key, d_value, k_cache, v_cache, d_slots, num_seqs, num_kv_heads, head_dim,
-                                      block_size, num_blocks, dtype, err_flags, stream);
-  if (st != PA_OK) return st;
-  st = pa_decode(d_out, d_q, k_cache, v_cache, d_tables, max_blocks_per_seq, d_ctx, num_seqs, max_context_len, scale,
-                 num_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype, workspace, workspace_bytes, 0,
-                 err_flags, stream);
+  const pa_status st = step_kernels(d_inputs, off, d_out, k_cache, v_cache, num_seqs, max_blocks_per_seq,
+                                    max_context_len, scale, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                    dtype, workspace, workspace_bytes, err_flags, stream);
   if (st != PA_OK) return st;
   const size_t out_bytes = static_cast<size_t>(num_seqs) * num_heads * head_dim * 2;
   e = cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host: device-to-host copy", e);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_decode_step_host_pipelined(const void* h_inputs, void* d_inputs, void* h_out, void* d_out,
+                                                   void* k_cache, void* v_cache, int num_seqs, int max_blocks_per_seq,
+                                                   int max_context_len, float scale, int num_heads, int num_kv_heads,
+                                                   int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                                                   void* workspace, size_t workspace_bytes, int32_t* err_flags,
+                                                   pa_stream_t stream, pa_stream_t copy_stream,
+                                                   pa_event_t inputs_ready, pa_event_t inputs_free) {
+  size_t off[6];
+  const size_t total = pa_step_inputs_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq, off);
+  if (total == 0) return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!h_inputs || !d_inputs || !h_out || !d_out || !inputs_ready || !inputs_free) return PA_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(d_inputs) & 255u) return PA_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+  cudaEvent_t ready = reinterpret_cast<cudaEvent_t>(inputs_ready);
+  cudaEvent_t free_ev = reinterpret_cast<cudaEvent_t>(inputs_free);
+  // The copy may start once the kernels of the last step that read this
+  // staging buffer are done (inputs_free, recorded by that step), not when
+  // the previous step's kernels are: it overlaps them.
+  cudaError_t e = cudaStreamWaitEvent(cs, free_ev, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_inputs, h_inputs, total, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaEventRecord(ready, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ready, 0);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host_pipelined: host-to-device copy", e);
+  const pa_status st = step_kernels(d_inputs, off, d_out, k_cache, v_cache, num_seqs, max_blocks_per_seq,
+                                    max_context_len, scale, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                    dtype, workspace, workspace_bytes, err_flags, stream);
+  if (st != PA_OK) return st;
+  e = cudaEventRecord(free_ev, s);  // this buffer's inputs are consumed
+  if (e == cudaSuccess) {
+    const size_t out_bytes = static_cast<size_t>(num_seqs) * num_heads * head_dim * 2;
+    e = cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, s);
+  }
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host_pipelined: device-to-host copy", e);
   return PA_OK;
 }

@@ -674,17 +674,25 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     const int64_t a = first ? af : al;
     const UnitPos& u = first ? uf : ul;
     const int mine = first ? mine_f : mine_l;
-    __threadfence();  // this lane's partial stores before the ticket
+    // Ordering without fences: the warp barrier orders every lane's partial
+    // stores before lane 0's ticket, whose release semantics publish them at
+    // GPU scope; the acquire half makes the other parts' partials (published
+    // the same way before their tickets) visible to lane 0, and the second
+    // barrier extends that to the lanes that read them.  (A __threadfence()
+    // on either side stalled each warp on its own loads in flight: ~3.5 us
+    // per launch on the LLaMA-7B workload.)
     __syncwarp();
     int last = 0;
     if (lane == 0) {
       int* t = p.ws_tickets + warp_of_chunk(a, NC, W);
-      const int before = atomicAdd(t, mine);
+      int before;
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(before) : "l"(t), "r"(mine) : "memory");
       last = before + mine == u.nc;
       if (last) *t = 0;  // all parts counted; nobody else touches it in this launch
     }
-    if (__shfl_sync(kFull, last, 0)) {
-      __threadfence();  // the other parts' stores, published before their tickets
+    last = __shfl_sync(kFull, last, 0);
+    __syncwarp();
+    if (last) {
       merge_split_unit<T, D, G>(p.ws_ml, p.ws_o,
                                 static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D, a,
                                 u.nc, NC, W, lane);

@@ -44,8 +44,8 @@ __device__ __forceinline__ void fold_partial(float& m, float& l, float4& acc, fl
 // Merge the partials of the unit of `nc` chunks starting at global chunk `a`
 // and write its G q-head rows (out_row -> [G][D]).  One warp; lane i owns
 // the float4 columns i, i+32, ... of the G*D outputs.  The partials were
-// written by other warps of this grid and published before their tickets
-// (the caller has fenced after drawing the last ticket), so they are read
+// written by other warps of this grid and published by their tickets'
+// release (the caller acquired them with the last ticket), so they are read
 // through L2 (ld.global.cg), never from a possibly stale L1 line.  A partial
 // whose running max is -inf (every token of that part skipped) adds nothing.
 template <typename T, int D, int G>

@@ -25,7 +25,7 @@ ERRF_CONTEXT = 1 << 2
 ERRF_TIMEOUT = 1 << 3
 
 SYMBOLS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_static",
-           "pa_decode_step_host", "pa_step_inputs_layout", "pa_prefill", "pa_prefill_mma", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
+           "pa_decode_step_host", "pa_decode_step_host_pipelined", "pa_step_inputs_layout", "pa_prefill", "pa_prefill_mma", "pa_copy_blocks", "pa_swap_blocks", "pa_bm_create",
            "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slot",
            "pa_bm_free_sequence", "pa_bm_context_len", "pa_bm_block_table", "pa_bm_blocks_needed_to_append",
            "pa_bm_prepare_decode", "pa_bm_swap_sequence", "pa_selftest_wait_timeout", "pa_selftest_exp2", "pa_status_string",
@@ -71,6 +71,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode_step_host.argtypes = [_vp] * 6 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64, _i32,
                                                     _vp, _sz, _vp, _vp]
     lib.pa_decode_step_host.restype = _i32
+    lib.pa_decode_step_host_pipelined.argtypes = [_vp] * 6 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64,
+                                                              _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp]
+    lib.pa_decode_step_host_pipelined.restype = _i32
     for f in ("pa_prefill", "pa_prefill_mma"):
         getattr(lib, f).argtypes = [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32,
                                     _i32, _i32, _i64, _i32, _vp, _vp]
@@ -272,6 +275,48 @@ def decode_step_host(h_inputs: torch.Tensor, d_inputs: torch.Tensor, h_out: torc
     if st != PA_OK:
         raise LibpagedError(st, "pa_decode_step_host")
     return h_out
+
+
+class StepPipeline:
+    """Host-driven decode steps with the input copy of step i+1 overlapping
+    the kernels of step i (pa_decode_step_host_pipelined): two device
+    staging buffers, each with its pair of events, used in turn, and a copy
+    stream beside the compute stream."""
+
+    def __init__(self, staging_bytes: int, device=None, stream=None, copy_stream=None):
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
+        self.copy_stream = copy_stream if copy_stream is not None else torch.cuda.Stream(dev)
+        self.d_inputs = [torch.empty(staging_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.events = [(torch.cuda.Event(), torch.cuda.Event()) for _ in range(2)]
+        for ready, free in self.events:  # creates the events (torch makes them on first record)
+            ready.record(self.stream)
+            free.record(self.stream)
+        self.step_index = 0
+
+    def step(self, h_inputs: torch.Tensor, h_out: torch.Tensor, d_out: torch.Tensor, k_cache: torch.Tensor,
+             v_cache: torch.Tensor, num_heads: int, max_blocks_per_seq: int, scale: float,
+             max_context_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+             err_flags: Optional[torch.Tensor] = None) -> torch.Tensor:
+        b = self.step_index % 2
+        self.step_index += 1
+        S = h_out.shape[0]
+        nb, kvh, bs, D = k_cache.shape
+        if max_context_len is None:
+            max_context_len = max_blocks_per_seq * bs
+        if workspace is None:
+            workspace = alloc_workspace(S, num_heads, kvh, D, max_context_len, device=k_cache.device)
+        ready, free = self.events[b]
+        st = load().pa_decode_step_host_pipelined(
+            _host_ptr(h_inputs, "h_inputs"), _dev_ptr(self.d_inputs[b], "d_inputs"), _host_ptr(h_out, "h_out"),
+            _dev_ptr(d_out, "d_out"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), S,
+            max_blocks_per_seq, int(max_context_len), float(scale), num_heads, kvh, D, bs, nb,
+            dtype_code(k_cache.dtype), _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            _dev_ptr(err_flags, "err_flags"), self.stream.cuda_stream, self.copy_stream.cuda_stream,
+            ready.cuda_event, free.cuda_event)
+        if st != PA_OK:
+            raise LibpagedError(st, "pa_decode_step_host_pipelined")
+        return h_out
 
 
 # ------------------------------------------------------------------ block operations

@@ -337,3 +337,52 @@ def test_merge_tickets_return_to_zero_and_workspace_reuse_is_exact():
             assert np.array_equal(got, want), (seed, max_ctas)
             assert int(shared[:nbytes].count_nonzero().item()) == 0, (seed, max_ctas)
         assert int(ds.err.item()) == 0
+
+
+def test_pipelined_host_steps_match_single_steps():
+    """pa_decode_step_host_pipelined (input copy of step i+1 on a second
+    stream, overlapping step i's kernels; two staging buffers in turn) gives,
+    step after step, the same bits as pa_decode_step_host."""
+    steps = []
+    for seed in (301, 302, 303, 304, 305):
+        steps.append(inputs.random_case(seed, num_seqs=6, num_heads=16, num_kv_heads=4, head_dim=128,
+                                        block_size=16, dtype="bf16", ctx_lo=1, ctx_hi=1500))
+    # one pool for all steps: each step's tables were drawn for its own pool,
+    # so use one workload's pool and tables and vary q and the new tokens
+    base = steps[0]
+    mb = base.max_blocks_per_seq
+    offs, total = libpaged.step_inputs_layout(base.num_seqs, base.num_heads, base.num_kv_heads, base.head_dim, mb)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+    h_ins = []
+    for wl in steps:
+        h = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        libpaged.pack_step_inputs(h, offs, q=t(wl.q), key=t(wl.k_new), value=t(wl.v_new),
+                                  slot_mapping=t(base.slot_mapping.astype(np.int64)),
+                                  block_tables=t(base.block_tables.astype(np.int32)),
+                                  context_lens=t(base.context_lens.astype(np.int32)))
+        h_ins.append(h)
+    want_state = DeviceState(base, full_pool=True)
+    got_state = DeviceState(base, full_pool=True)
+    d_in = torch.empty(total, dtype=torch.uint8, device="cuda")
+    pipe = libpaged.StepPipeline(total)
+    want, got = [], []
+    for h in h_ins:
+        ho = torch.empty(want_state.q.shape, dtype=torch.bfloat16).pin_memory()
+        libpaged.decode_step_host(h, d_in, ho, torch.empty_like(want_state.q), want_state.k_cache,
+                                  want_state.v_cache, base.num_heads, mb, float(base.scale),
+                                  max_context_len=base.max_context_len, workspace=want_state.ws,
+                                  err_flags=want_state.err)
+        torch.cuda.synchronize()
+        want.append(ho.clone())
+    outs = []
+    for h in h_ins:
+        ho = torch.empty(got_state.q.shape, dtype=torch.bfloat16).pin_memory()
+        pipe.step(h, ho, torch.empty_like(got_state.q), got_state.k_cache, got_state.v_cache, base.num_heads, mb,
+                  float(base.scale), max_context_len=base.max_context_len, workspace=got_state.ws,
+                  err_flags=got_state.err)
+        outs.append(ho)
+    torch.cuda.synchronize()
+    for a, b in zip(want, outs):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(want_state.k_cache.view(torch.int16), got_state.k_cache.view(torch.int16))
+    assert int(got_state.err.item()) == 0
