@@ -14,6 +14,7 @@
 // buffers used in turn, so that it overlaps the previous step's kernels
 // instead of preceding them.
 #include "pa_device.cuh"
+#include "pa_host.h"
 
 namespace {
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -70,10 +71,14 @@ extern "C" pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, v
                                          int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
                                          void* workspace, size_t workspace_bytes, int32_t* err_flags,
                                          pa_stream_t stream) {
+  pa::DecodePlan plan;  // the decode's argument checks, before anything is enqueued
+  const pa_status pst = pa::plan_decode(num_seqs, max_blocks_per_seq, max_context_len, scale, num_heads,
+                                        num_kv_heads, head_dim, block_size, num_blocks, dtype, 0, &plan);
+  if (pst != PA_OK) return pst;
+  if (num_seqs == 0) return PA_OK;
   size_t off[6];
   const size_t total = pa_step_inputs_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq, off);
   if (total == 0) return PA_ERR_INVALID;
-  if (num_seqs == 0) return PA_OK;
   if (!h_inputs || !d_inputs || !h_out || !d_out) return PA_ERR_INVALID;
   if (reinterpret_cast<uintptr_t>(d_inputs) & 255u) return PA_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -96,10 +101,14 @@ extern "C" pa_status pa_decode_step_host_pipelined(const void* h_inputs, void* d
                                                    void* workspace, size_t workspace_bytes, int32_t* err_flags,
                                                    pa_stream_t stream, pa_stream_t copy_stream,
                                                    pa_event_t inputs_ready, pa_event_t inputs_free) {
+  pa::DecodePlan plan;  // the decode's argument checks, before anything is enqueued
+  const pa_status pst = pa::plan_decode(num_seqs, max_blocks_per_seq, max_context_len, scale, num_heads,
+                                        num_kv_heads, head_dim, block_size, num_blocks, dtype, 0, &plan);
+  if (pst != PA_OK) return pst;
+  if (num_seqs == 0) return PA_OK;
   size_t off[6];
   const size_t total = pa_step_inputs_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq, off);
   if (total == 0) return PA_ERR_INVALID;
-  if (num_seqs == 0) return PA_OK;
   if (!h_inputs || !d_inputs || !h_out || !d_out || !inputs_ready || !inputs_free) return PA_ERR_INVALID;
   if (reinterpret_cast<uintptr_t>(d_inputs) & 255u) return PA_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

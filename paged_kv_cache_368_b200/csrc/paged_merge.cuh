@@ -29,81 +29,124 @@ __device__ __forceinline__ int64_t partial_slot(int64_t w, int64_t a, int64_t NC
   return 2 * w + (run_begin(w, NC, W) >= a ? 0 : 1);
 }
 
-// One online-softmax fold of a partial (ml = (m, l), o) into (m, l, acc).
-__device__ __forceinline__ void fold_partial(float& m, float& l, float4& acc, float2 ml, float4 o) {
-  const float mn = fmaxf(m, ml.x);
-  const float sa = fast_exp2(m - mn), sb = fast_exp2(ml.x - mn);
-  l = l * sa + ml.y * sb;
-  acc.x = acc.x * sa + o.x * sb;
-  acc.y = acc.y * sa + o.y * sb;
-  acc.z = acc.z * sa + o.z * sb;
-  acc.w = acc.w * sa + o.w * sb;
-  m = mn;
-}
-
 // Merge the partials of the unit of `nc` chunks starting at global chunk `a`
-// and write its G q-head rows (out_row -> [G][D]).  One warp; lane i owns
-// the float4 columns i, i+32, ... of the G*D outputs.  The partials were
-// written by other warps of this grid and published by their tickets'
-// release (the caller acquired them with the last ticket), so they are read
-// through L2 (ld.global.cg), never from a possibly stale L1 line.  A partial
-// whose running max is -inf (every token of that part skipped) adds nothing.
+// and write its G q-head rows (out_row -> [G][D]).  One warp, two phases per
+// block of up to 32 contributors:
+//  1. lane j reads contributor j's (m, l) for every q-head; warp reductions
+//     give the block's maximum M_g and each contributor's weight
+//     2^(m_jg - M_g) (folded into the running maximum of earlier blocks);
+//  2. lane i owns the float4 output columns i, i+32, ... and adds up
+//     weight * o over the block's contributors.  The weights are known, so
+//     the loads of several contributors are independent and in flight
+//     together (up to 16 float4 columns per lane), instead of one round trip
+//     per contributor.
+// The partials were written by other warps of this grid and published by
+// their tickets' release (the caller acquired them with the last ticket), so
+// they are read through L2 (ld.global.cg), never from a possibly stale L1
+// line.  A partial whose running max is -inf (every token of that part
+// skipped) has weight 0.
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_split_unit(const float2* ws_ml, const float* ws_o, T* out_row, int64_t a,
                                                  int nc, int64_t NC, int W, int lane) {
   using E = Elem<T>;
-  constexpr int kItems = G * D / 4;                   // float4 outputs
+  constexpr int kItems = G * D / 4;          // float4 outputs
   constexpr int kPerLane = (kItems + 31) / 32;
-  // contributors loaded before folding: about eight float4 columns in flight
-  // per lane, whatever G (the merge runs inside the streaming loop and its
-  // registers add to the loop's)
-  constexpr int kBatch = kPerLane >= 8 ? 1 : 8 / kPerLane;
+  constexpr int kBatch = kPerLane >= 8 ? 1 : 4;  // contributors in flight in phase 2
+  constexpr int kHeadItems = D / 4;          // float4 columns of one q-head
   const int w0 = warp_of_chunk(a, NC, W);
-  const int w1 = warp_of_chunk(a + nc - 1, NC, W);
-  float m[kPerLane], l[kPerLane];
+  const int nw = warp_of_chunk(a + nc - 1, NC, W) - w0 + 1;
+  float M[G], L[G];  // running maximum (log2 units) and weighted sum of l, per q-head
   float4 acc[kPerLane];
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    m[i] = -INFINITY;
-    l[i] = 0.f;
-    acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int g = 0; g < G; ++g) {
+    M[g] = -INFINITY;
+    L[g] = 0.f;
   }
-  for (int w = w0; w <= w1; w += kBatch) {
-    float2 ml[kBatch][kPerLane];
-    float4 o[kBatch][kPerLane];
-    bool use[kBatch];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int wu = w + u;
-      // Warps with an empty run (more warps than chunks) wrote nothing.
-      use[u] = wu <= w1 && run_begin(wu, NC, W) < run_begin(wu + 1, NC, W);
-      const int64_t slot = use[u] ? partial_slot(wu, a, NC, W) : 0;
+  for (int i = 0; i < kPerLane; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+  for (int base = 0; base < nw; base += 32) {
+    // ---- phase 1: this lane's contributor of the block
+    const int wj = w0 + base + lane;
+    // Warps with an empty run (more warps than chunks) wrote nothing.
+    const bool has = base + lane < nw && run_begin(wj, NC, W) < run_begin(wj + 1, NC, W);
+    const int slot = has ? static_cast<int>(partial_slot(wj, a, NC, W)) : 0;
+    float wgt[G];
 #pragma unroll
-      for (int i = 0; i < kPerLane; ++i) {
-        const int item = lane + 32 * i;
-        const int g = item / (D / 4), d4 = item % (D / 4);
-        if (use[u] && item < kItems) {
-          ml[u][i] = __ldcg(ws_ml + slot * G + g);
-          o[u][i] = __ldcg(reinterpret_cast<const float4*>(ws_o + (slot * G + g) * D) + d4);
-        } else {
-          ml[u][i] = make_float2(-INFINITY, 0.f);
-          o[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = 0; g < G; ++g) {
+      const float2 ml = has ? __ldcg(ws_ml + (int64_t)slot * G + g) : make_float2(-INFINITY, 0.f);
+      float mb = ml.x;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
+      const float mn = fmaxf(M[g], mb);
+      // rescale what earlier blocks accumulated for this head to the new maximum
+      const float rs = M[g] == -INFINITY ? 0.f : fast_exp2(M[g] - mn);
+      if (rs != 1.f) {
+        L[g] *= rs;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+          if ((lane + 32 * i) / kHeadItems == g) {
+            acc[i].x *= rs;
+            acc[i].y *= rs;
+            acc[i].z *= rs;
+            acc[i].w *= rs;
+          }
         }
       }
+      M[g] = mn;
+      wgt[g] = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mn);
+      float ls = wgt[g] * ml.y;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
+      L[g] += ls;
     }
+    // ---- phase 2: weighted sum of the block's partial outputs
+    const int nb = min(32, nw - base);
+    for (int j = 0; j < nb; j += kBatch) {
+      float4 o[kBatch][kPerLane];
+      float wv[kBatch][kPerLane];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
+      for (int u = 0; u < kBatch; ++u) {
+        const int src = min(j + u, 31);
+        const bool use = j + u < nb && __shfl_sync(kFull, has, src);
+        const int sl = __shfl_sync(kFull, slot, src);
+        float wg[G];
 #pragma unroll
-      for (int i = 0; i < kPerLane; ++i)
-        if (ml[u][i].x != -INFINITY) fold_partial(m[i], l[i], acc[i], ml[u][i], o[u][i]);
+        for (int g = 0; g < G; ++g) wg[g] = __shfl_sync(kFull, wgt[g], src);
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+          const int item = lane + 32 * i;
+          const int g = item / kHeadItems, d4 = item % kHeadItems;
+          float w = 0.f;
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) w = gg == g ? wg[gg] : w;
+          wv[u][i] = use ? w : 0.f;
+          o[u][i] = (use && item < kItems && w != 0.f)
+                        ? __ldcg(reinterpret_cast<const float4*>(ws_o + ((int64_t)sl * G + g) * D) + d4)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+          acc[i].x = fmaf(wv[u][i], o[u][i].x, acc[i].x);
+          acc[i].y = fmaf(wv[u][i], o[u][i].y, acc[i].y);
+          acc[i].z = fmaf(wv[u][i], o[u][i].z, acc[i].z);
+          acc[i].w = fmaf(wv[u][i], o[u][i].w, acc[i].w);
+        }
+      }
     }
   }
 #pragma unroll
   for (int i = 0; i < kPerLane; ++i) {
     const int item = lane + 32 * i;
     if (item >= kItems) continue;
-    const int g = item / (D / 4), d4 = item % (D / 4);
-    const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
+    const int g = item / kHeadItems, d4 = item % kHeadItems;
+    float lg = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) lg = gg == g ? L[gg] : lg;
+    const float inv = lg > 0.f ? 1.f / lg : 0.f;
     uint2 u;
     u.x = E::pack(acc[i].x * inv, acc[i].y * inv);
     u.y = E::pack(acc[i].z * inv, acc[i].w * inv);

@@ -31,6 +31,7 @@
 #include <atomic>
 #include <cmath>
 
+#include "exp2_poly.cuh"
 #include "pa_host.h"
 #include "tcgen05.cuh"
 
@@ -41,6 +42,16 @@ constexpr int BM = 128;  // query rows per softmax group (MMA M)
 constexpr int BN = 64;   // keys per tile (MMA N of S, K of P.V)
 constexpr int kGroups = 2;  // query tiles (softmax warpgroups) per CTA sharing each K/V tile
 constexpr uint64_t kWaitNs = 1000000000ull;
+
+// Which exponentials of the softmax run as the FMA-pipe polynomial of
+// exp2_poly.cuh (two at a time) instead of on the special-function unit:
+// bit b of the mask set -> the key pairs 8m+b.
+#ifndef PA_PREFILL_POLY_MASK_D128
+#define PA_PREFILL_POLY_MASK_D128 0x00  // none: measured 908 vs 917 TFLOP/s with 1/8
+#endif
+#ifndef PA_PREFILL_POLY_MASK_D64
+#define PA_PREFILL_POLY_MASK_D64 0x88   // pairs 3 and 7 of 8: 1/4 (547 vs 513 TFLOP/s)
+#endif
 
 
 struct Params {
@@ -76,6 +87,8 @@ struct Lay {
   static constexpr int kBars = 1 + 2 * STAGES + NWG * 6 + 1;
   static constexpr size_t kSmem = 1024 + kOffBar + kBars * 8 + 16;
   static constexpr int kThreads = (4 + 4 * NWG) * 32;  // warps 0-3: TMA (Q, K), MMA, TMA (V), idle
+  // key pairs 8m+b with bit b set take the FMA-pipe polynomial for their exponentials
+  static constexpr unsigned kPolyMask = D == 128 ? PA_PREFILL_POLY_MASK_D128 : PA_PREFILL_POLY_MASK_D64;
   // Tensor memory per group: S0 | S1 | O.  P of tile j (16-bit, two per
   // column) overwrites the front of S(j & 1) once the softmax has read it.
   static constexpr uint32_t kColsPerGroup = 2 * BN + D;
@@ -429,9 +442,14 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
       float ls[4][2] = {};
 #pragma unroll
       for (int i = 0; i < BN / 2; ++i) {
-        float x0, x1;
+        float x0, x1, p0, p1;
         tc5::fma2(x0, x1, sv[2 * i], sv[2 * i + 1], p.scale_log2, -mref);
-        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        if ((L::kPolyMask >> (i & 7)) & 1u) {
+          exp2_poly2(p0, p1, x0, x1);
+        } else {
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
+        }
         tc5::add2(ls[i & 3][0], ls[i & 3][1], p0, p1);
         pk[i] = E::pack(p0, p1);
       }
