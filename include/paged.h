@@ -166,29 +166,38 @@ PA_API pa_status pa_decode_step_host(const void* h_inputs, void* d_inputs, void*
 
 /*
  * pa_decode_step_host_pipelined -- pa_decode_step_host for a loop of decode
- * steps, with each step's host-to-device copy overlapping the previous
- * step's kernels.  The copy of h_inputs into d_inputs is enqueued on
- * copy_stream; append, decode and the copy of the output into h_out on
- * `stream`, after the input copy (event inputs_ready).  The caller keeps two
- * staging buffers, each 256-byte aligned and pa_step_inputs_layout() bytes,
- * with a pair of events of its own (created by the caller, e.g. with
- * cudaEventCreateWithFlags(..., cudaEventDisableTiming)), and passes them in
- * turn: step i uses buffer i % 2 with its events.  A buffer's copy waits
- * (inputs_free) only until the kernels of the step that last read it have
- * finished, two steps earlier, so it runs while step i-1 computes.  h_out is
- * valid once `stream` reaches the end of the call; h_inputs must stay
- * unchanged until the copy has run (inputs_ready), so alternate two host
- * buffers as well when they are refilled every step.  A never-recorded
- * inputs_free makes the first copy start at once.  Errors as for
- * pa_decode_step_host; PA_ERR_INVALID for a NULL event.
+ * steps, with each step's copies overlapping the neighbouring steps' kernels.
+ * Three streams take part:
+ *   in_stream   the copy h_inputs -> d_inputs, then event inputs_ready;
+ *   stream      append and decode into d_out, after inputs_ready and after
+ *               output_free (the previous copy out of this d_out); then
+ *               events inputs_free and output_ready;
+ *   out_stream  the copy d_out -> h_out after output_ready, then event
+ *               output_free.
+ * The caller keeps two sets of {d_inputs (256-byte aligned,
+ * pa_step_inputs_layout() bytes), d_out, inputs_ready, inputs_free,
+ * output_ready, output_free} and passes them in turn: step i uses set i % 2.
+ * A set's input copy waits only until the kernels that last read its
+ * d_inputs (two steps earlier) are done, so it runs while step i-1 computes;
+ * its output copy runs while step i+1 computes.  The events are the
+ * caller's (e.g. cudaEventCreateWithFlags(..., cudaEventDisableTiming)); a
+ * never-recorded event counts as complete, so the first steps start at once.
+ * The copies overlap the kernels only when the three streams are distinct;
+ * the results are the same either way.  h_out holds step i's output once
+ * output_free of step i has completed (cudaEventSynchronize, or a
+ * cudaStreamWaitEvent before a consumer); h_inputs must stay unchanged until
+ * inputs_ready has completed, so alternate two host buffers as well when they
+ * are refilled every step.  Errors as for pa_decode_step_host; PA_ERR_INVALID
+ * for a NULL event.
  */
 PA_API pa_status pa_decode_step_host_pipelined(const void* h_inputs, void* d_inputs, void* h_out, void* d_out,
                                                void* k_cache, void* v_cache, int num_seqs, int max_blocks_per_seq,
                                                int max_context_len, float scale, int num_heads, int num_kv_heads,
                                                int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
                                                void* workspace, size_t workspace_bytes, int32_t* err_flags,
-                                               pa_stream_t stream, pa_stream_t copy_stream, pa_event_t inputs_ready,
-                                               pa_event_t inputs_free);
+                                               pa_stream_t stream, pa_stream_t in_stream, pa_stream_t out_stream,
+                                               pa_event_t inputs_ready, pa_event_t inputs_free,
+                                               pa_event_t output_ready, pa_event_t output_free);
 
 /*
  * pa_decode_static -- pa_decode for callers that cannot allocate device

@@ -12,7 +12,10 @@
 // pa_decode_step_host_pipelined is the same step for a serving loop: its
 // host-to-device copy runs on a second stream, into one of two staging
 // buffers used in turn, so that it overlaps the previous step's kernels
-// instead of preceding them.
+// instead of preceding them; its device-to-host copy runs on a third, out of
+// one of two output buffers, so that it overlaps the next step's kernels.
+// A copy between two kernels on one stream also ends the programmatic-launch
+// overlap of their start and end, which costs more than the copy itself.
 #include "pa_device.cuh"
 #include "pa_host.h"
 
@@ -99,8 +102,9 @@ extern "C" pa_status pa_decode_step_host_pipelined(const void* h_inputs, void* d
                                                    int max_context_len, float scale, int num_heads, int num_kv_heads,
                                                    int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
                                                    void* workspace, size_t workspace_bytes, int32_t* err_flags,
-                                                   pa_stream_t stream, pa_stream_t copy_stream,
-                                                   pa_event_t inputs_ready, pa_event_t inputs_free) {
+                                                   pa_stream_t stream, pa_stream_t in_stream, pa_stream_t out_stream,
+                                                   pa_event_t inputs_ready, pa_event_t inputs_free,
+                                                   pa_event_t output_ready, pa_event_t output_free) {
   pa::DecodePlan plan;  // the decode's argument checks, before anything is enqueued
   const pa_status pst = pa::plan_decode(num_seqs, max_blocks_per_seq, max_context_len, scale, num_heads,
                                         num_kv_heads, head_dim, block_size, num_blocks, dtype, 0, &plan);
@@ -109,29 +113,43 @@ extern "C" pa_status pa_decode_step_host_pipelined(const void* h_inputs, void* d
   size_t off[6];
   const size_t total = pa_step_inputs_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq, off);
   if (total == 0) return PA_ERR_INVALID;
-  if (!h_inputs || !d_inputs || !h_out || !d_out || !inputs_ready || !inputs_free) return PA_ERR_INVALID;
+  if (!h_inputs || !d_inputs || !h_out || !d_out) return PA_ERR_INVALID;
+  if (!inputs_ready || !inputs_free || !output_ready || !output_free) return PA_ERR_INVALID;
   if (reinterpret_cast<uintptr_t>(d_inputs) & 255u) return PA_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
-  cudaEvent_t ready = reinterpret_cast<cudaEvent_t>(inputs_ready);
-  cudaEvent_t free_ev = reinterpret_cast<cudaEvent_t>(inputs_free);
-  // The copy may start once the kernels of the last step that read this
-  // staging buffer are done (inputs_free, recorded by that step), not when
-  // the previous step's kernels are: it overlaps them.
-  cudaError_t e = cudaStreamWaitEvent(cs, free_ev, 0);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(d_inputs, h_inputs, total, cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess) e = cudaEventRecord(ready, cs);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ready, 0);
+  cudaStream_t is = reinterpret_cast<cudaStream_t>(in_stream);
+  cudaStream_t os = reinterpret_cast<cudaStream_t>(out_stream);
+  cudaEvent_t in_ready = reinterpret_cast<cudaEvent_t>(inputs_ready);
+  cudaEvent_t in_free = reinterpret_cast<cudaEvent_t>(inputs_free);
+  cudaEvent_t out_ready = reinterpret_cast<cudaEvent_t>(output_ready);
+  cudaEvent_t out_free = reinterpret_cast<cudaEvent_t>(output_free);
+  // Input copy: once the kernels of the last step that read this staging
+  // buffer are done (not the previous step's: it overlaps them).
+  cudaError_t e = cudaStreamWaitEvent(is, in_free, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_inputs, h_inputs, total, cudaMemcpyHostToDevice, is);
+  if (e == cudaSuccess) e = cudaEventRecord(in_ready, is);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host_pipelined: host-to-device copy", e);
+  // Kernels: after this step's inputs and after the copy out of this d_out
+  // two steps back.  Both waits come before the append, so nothing sits
+  // between the append and the decode, which overlap through the
+  // programmatic launch.
+  e = cudaStreamWaitEvent(s, in_ready, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, out_free, 0);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host_pipelined: stream wait", e);
   const pa_status st = step_kernels(d_inputs, off, d_out, k_cache, v_cache, num_seqs, max_blocks_per_seq,
                                     max_context_len, scale, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                     dtype, workspace, workspace_bytes, err_flags, stream);
   if (st != PA_OK) return st;
-  e = cudaEventRecord(free_ev, s);  // this buffer's inputs are consumed
+  e = cudaEventRecord(in_free, s);  // this buffer's inputs are consumed
+  if (e == cudaSuccess) e = cudaEventRecord(out_ready, s);
+  // Output copy, off the compute stream: the next step's kernels start
+  // without waiting for it.
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(os, out_ready, 0);
   if (e == cudaSuccess) {
     const size_t out_bytes = static_cast<size_t>(num_seqs) * num_heads * head_dim * 2;
-    e = cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, os);
   }
+  if (e == cudaSuccess) e = cudaEventRecord(out_free, os);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step_host_pipelined: device-to-host copy", e);
   return PA_OK;
 }

@@ -72,7 +72,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
                                                     _vp, _sz, _vp, _vp]
     lib.pa_decode_step_host.restype = _i32
     lib.pa_decode_step_host_pipelined.argtypes = [_vp] * 6 + [_i32, _i32, _i32, _f32, _i32, _i32, _i32, _i32, _i64,
-                                                              _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp]
+                                                              _i32, _vp, _sz, _vp] + [_vp] * 7
     lib.pa_decode_step_host_pipelined.restype = _i32
     for f in ("pa_prefill", "pa_prefill_mma"):
         getattr(lib, f).argtypes = [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _f32, _i32, _i32,
@@ -278,26 +278,46 @@ def decode_step_host(h_inputs: torch.Tensor, d_inputs: torch.Tensor, h_out: torc
 
 
 class StepPipeline:
-    """Host-driven decode steps with the input copy of step i+1 overlapping
-    the kernels of step i (pa_decode_step_host_pipelined): two device
-    staging buffers, each with its pair of events, used in turn, and a copy
-    stream beside the compute stream."""
+    """Host-driven decode steps whose copies overlap the neighbouring steps'
+    kernels (pa_decode_step_host_pipelined): the input copy of step i+1 runs
+    on ``in_stream`` while step i computes, the output copy of step i on
+    ``out_stream`` while step i+1 computes.  Two sets of device staging
+    buffer, device output buffer and four events are used in turn."""
 
-    def __init__(self, staging_bytes: int, device=None, stream=None, copy_stream=None):
+    def __init__(self, staging_bytes: int, out_shape, dtype: torch.dtype, device=None, stream=None, in_stream=None,
+                 out_stream=None):
         dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
-        self.copy_stream = copy_stream if copy_stream is not None else torch.cuda.Stream(dev)
+        self.in_stream = in_stream if in_stream is not None else torch.cuda.Stream(dev)
+        self.out_stream = out_stream if out_stream is not None else torch.cuda.Stream(dev)
         self.d_inputs = [torch.empty(staging_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-        self.events = [(torch.cuda.Event(), torch.cuda.Event()) for _ in range(2)]
-        for ready, free in self.events:  # creates the events (torch makes them on first record)
-            ready.record(self.stream)
-            free.record(self.stream)
+        self.d_out = [torch.empty(tuple(out_shape), dtype=dtype, device=dev) for _ in range(2)]
+        # per set: inputs_ready, inputs_free, output_ready, output_free
+        self.events = [tuple(torch.cuda.Event() for _ in range(4)) for _ in range(2)]
+        for evs in self.events:  # creates the events (torch makes them on first record)
+            for ev in evs:
+                ev.record(self.stream)
         self.step_index = 0
 
-    def step(self, h_inputs: torch.Tensor, h_out: torch.Tensor, d_out: torch.Tensor, k_cache: torch.Tensor,
-             v_cache: torch.Tensor, num_heads: int, max_blocks_per_seq: int, scale: float,
-             max_context_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
-             err_flags: Optional[torch.Tensor] = None) -> torch.Tensor:
+    def args(self, b: int, h_inputs: torch.Tensor, h_out: torch.Tensor, k_cache: torch.Tensor,
+             v_cache: torch.Tensor, num_heads: int, max_blocks_per_seq: int, scale: float, max_context_len: int,
+             workspace: torch.Tensor, err_flags: Optional[torch.Tensor] = None) -> tuple:
+        """The C-ABI arguments of a step that uses set ``b`` (built once and
+        reused by a loop that calls the library directly)."""
+        S = h_out.shape[0]
+        nb, kvh, bs, D = k_cache.shape
+        return (_host_ptr(h_inputs, "h_inputs"), _dev_ptr(self.d_inputs[b], "d_inputs"), _host_ptr(h_out, "h_out"),
+                _dev_ptr(self.d_out[b], "d_out"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), S,
+                max_blocks_per_seq, int(max_context_len), float(scale), num_heads, kvh, D, bs, nb,
+                dtype_code(k_cache.dtype), _dev_ptr(workspace, "workspace"),
+                workspace.numel() * workspace.element_size(), _dev_ptr(err_flags, "err_flags"),
+                self.stream.cuda_stream, self.in_stream.cuda_stream, self.out_stream.cuda_stream,
+                *(ev.cuda_event for ev in self.events[b]))
+
+    def step(self, h_inputs: torch.Tensor, h_out: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+             num_heads: int, max_blocks_per_seq: int, scale: float, max_context_len: Optional[int] = None,
+             workspace: Optional[torch.Tensor] = None, err_flags: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Enqueue one step; ``h_out`` holds its output after ``wait()``."""
         b = self.step_index % 2
         self.step_index += 1
         S = h_out.shape[0]
@@ -306,17 +326,24 @@ class StepPipeline:
             max_context_len = max_blocks_per_seq * bs
         if workspace is None:
             workspace = alloc_workspace(S, num_heads, kvh, D, max_context_len, device=k_cache.device)
-        ready, free = self.events[b]
-        st = load().pa_decode_step_host_pipelined(
-            _host_ptr(h_inputs, "h_inputs"), _dev_ptr(self.d_inputs[b], "d_inputs"), _host_ptr(h_out, "h_out"),
-            _dev_ptr(d_out, "d_out"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), S,
-            max_blocks_per_seq, int(max_context_len), float(scale), num_heads, kvh, D, bs, nb,
-            dtype_code(k_cache.dtype), _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-            _dev_ptr(err_flags, "err_flags"), self.stream.cuda_stream, self.copy_stream.cuda_stream,
-            ready.cuda_event, free.cuda_event)
+        st = load().pa_decode_step_host_pipelined(*self.args(b, h_inputs, h_out, k_cache, v_cache, num_heads,
+                                                             max_blocks_per_seq, scale, max_context_len, workspace,
+                                                             err_flags))
         if st != PA_OK:
             raise LibpagedError(st, "pa_decode_step_host_pipelined")
         return h_out
+
+    def join(self, stream=None) -> None:
+        """Make ``stream`` (default: the compute stream) wait for every copy
+        enqueued so far, without blocking the host."""
+        s = stream if stream is not None else self.stream
+        s.wait_stream(self.in_stream)
+        s.wait_stream(self.out_stream)
+
+    def wait(self) -> None:
+        """Block the host until the last step's output copy has landed."""
+        if self.step_index:
+            self.events[(self.step_index - 1) % 2][3].synchronize()
 
 
 # ------------------------------------------------------------------ block operations

@@ -104,14 +104,17 @@ def test_pipelined_step_host_checks(lib):
 
     def call(**kw):
         a = dict(h_in=16, d_in=256, h_out=16, d_out=16, kc=16, vc=16, S=2, mb=4, maxctx=64, scale=0.1, H=4, KVH=4,
-                 D=128, BS=16, NB=8, dt=0, ws=16, wsb=1 << 20, err=None, s=None, cs=None, ready=16, free=16)
+                 D=128, BS=16, NB=8, dt=0, ws=16, wsb=1 << 20, err=None, s=None, ins=None, outs=None, ready=16,
+                 free=16, oready=16, ofree=16)
         a.update(kw)
         return f(a["h_in"], a["d_in"], a["h_out"], a["d_out"], a["kc"], a["vc"], a["S"], a["mb"], a["maxctx"],
                  a["scale"], a["H"], a["KVH"], a["D"], a["BS"], a["NB"], a["dt"], a["ws"], a["wsb"], a["err"], a["s"],
-                 a["cs"], a["ready"], a["free"])
+                 a["ins"], a["outs"], a["ready"], a["free"], a["oready"], a["ofree"])
 
     assert call(ready=None) == I
     assert call(free=None) == I
+    assert call(oready=None) == I
+    assert call(ofree=None) == I
     assert call(h_in=None) == I
     assert call(d_in=264) == I  # staging buffer not 256-byte aligned
     assert call(H=6, KVH=4) == I

@@ -341,8 +341,10 @@ def test_merge_tickets_return_to_zero_and_workspace_reuse_is_exact():
 
 def test_pipelined_host_steps_match_single_steps():
     """pa_decode_step_host_pipelined (input copy of step i+1 on a second
-    stream, overlapping step i's kernels; two staging buffers in turn) gives,
-    step after step, the same bits as pa_decode_step_host."""
+    stream, overlapping step i's kernels; output copy of step i on a third,
+    overlapping step i+1's; two sets of staging and output buffers in turn,
+    so steps 0, 2 and 4 reuse one device output buffer) gives, step after
+    step, the same bits as pa_decode_step_host."""
     steps = []
     for seed in (301, 302, 303, 304, 305):
         steps.append(inputs.random_case(seed, num_seqs=6, num_heads=16, num_kv_heads=4, head_dim=128,
@@ -364,7 +366,7 @@ def test_pipelined_host_steps_match_single_steps():
     want_state = DeviceState(base, full_pool=True)
     got_state = DeviceState(base, full_pool=True)
     d_in = torch.empty(total, dtype=torch.uint8, device="cuda")
-    pipe = libpaged.StepPipeline(total)
+    pipe = libpaged.StepPipeline(total, got_state.q.shape, torch.bfloat16)
     want, got = [], []
     for h in h_ins:
         ho = torch.empty(want_state.q.shape, dtype=torch.bfloat16).pin_memory()
@@ -377,11 +379,10 @@ def test_pipelined_host_steps_match_single_steps():
     outs = []
     for h in h_ins:
         ho = torch.empty(got_state.q.shape, dtype=torch.bfloat16).pin_memory()
-        pipe.step(h, ho, torch.empty_like(got_state.q), got_state.k_cache, got_state.v_cache, base.num_heads, mb,
-                  float(base.scale), max_context_len=base.max_context_len, workspace=got_state.ws,
-                  err_flags=got_state.err)
+        pipe.step(h, ho, got_state.k_cache, got_state.v_cache, base.num_heads, mb, float(base.scale),
+                  max_context_len=base.max_context_len, workspace=got_state.ws, err_flags=got_state.err)
         outs.append(ho)
-    torch.cuda.synchronize()
+    pipe.wait()  # the last output copy; the earlier ones ran before it on the same stream
     for a, b in zip(want, outs):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert torch.equal(want_state.k_cache.view(torch.int16), got_state.k_cache.view(torch.int16))
