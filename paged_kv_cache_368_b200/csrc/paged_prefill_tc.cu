@@ -284,14 +284,34 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     }
   } else if (active && warp == 1) {
     // ------------------------------------------------------------- MMA issue
-    // The whole warp follows the schedule (so descriptors stay warp-uniform);
-    // one elected lane issues every MMA and commit.  Per tile j and group g:
-    // P.V of tile j, then the scores of tile j+2 into the S buffer that P
-    // occupied (tensor-core operations of one thread run in issue order).
+    // The whole warp follows the schedule, converged, and one elected lane
+    // issues every MMA and commit under a predicate (issuing from a lane
+    // that has diverged from its warp measured ~4x slower per MMA).  The
+    // warp shares its scheduler with two softmax warps and paces the tensor
+    // pipe, so its instruction count per tile matters: descriptors and tile
+    // counts are computed once, and each MMA only adds a constant offset.
+    // Per tile j, per query tile g: P.V of tile j, then the scores of tile
+    // j+2 into the S buffer that P occupied (tensor-core operations of one
+    // thread run in issue order).
     constexpr int fmt = Elem<T>::kind == PA_BF16 ? 1 : 0;
     constexpr uint32_t id_qk = tc5::f16_idesc(fmt, BM, BN, 0, 0);
     constexpr uint32_t id_pv = tc5::f16_idesc(fmt, BM, D, 0, 1);
     const uint32_t leader = tc5::elect_one();
+    // V tile, chunk-major: the head_dim halves of a chunk are box_rows * 128 B
+    // apart (LBO) and its two 8-key row groups 1 KB apart, or one block's box
+    // apart when a chunk spans two 8-row blocks (SBO).
+    const int box_rows = p.block_size < 16 ? p.block_size : 16;
+    const uint32_t v_lbo = box_rows * 128;
+    const uint32_t v_sbo = p.block_size >= 16 ? 1024u : uint32_t(D / 64) * 1024u;
+    // Descriptors of the first operand tiles; the offsets added below are in
+    // the descriptor's 16-byte units (the start-address field never carries:
+    // shared memory ends below 2^18 bytes).
+    const uint64_t dq = tc5::sw128_desc(q_s, 16, 1024);
+    const uint64_t dk = tc5::sw128_desc(k_s, 16, 1024);
+    const uint64_t dv = tc5::sw128_desc(v_s, v_lbo, v_sbo);
+    static_assert(NWG == 2, "two query tiles per CTA");
+    const int gt0 = g_tiles(0), gt1 = g_tiles(1);
+    auto gt = [&](int g) { return g == 0 ? gt0 : gt1; };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
       // one plain probe first: most of these waits are already satisfied,
       // and the suspending form costs the pacing warp ~100 cycles even then
@@ -301,44 +321,35 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     int kv_seen = -1;  // highest tile whose copies this warp has already waited for
     auto issue_qk = [&](int g, int j) -> bool {  // S(g, j&1) = Q_g K_j^T
       const int st = j % STAGES;
-      // Tiles are waited for in increasing order; the second group's scores
-      // of the same tile skip the (already satisfied) wait.
+      // Tiles are waited for in increasing order; the second query tile's
+      // scores of the same tile skip the (already satisfied) wait.
       if (j > kv_seen) {
         if (!wait_all(&kv_full[st], (j / STAGES) & 1)) return false;
         kv_seen = j;
       }
       tc5::fence_after();
-      const uint32_t kt = k_s + st * L::kKV, qt = q_s + g * L::kQ;
+      const uint64_t a = dq + uint64_t(g * (L::kQ >> 4));
+      const uint64_t b = dk + uint64_t(st * (L::kKV >> 4));
       const uint32_t sd = tmem + g * L::kColsPerGroup + (j & 1) * BN;
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint64_t da = tc5::sw128_desc(qt + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024);
-        const uint64_t db = tc5::sw128_desc(kt + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024);
-        tc5::mma_ss_if(leader, sd, da, db, id_qk, ks > 0);
-      }
+      for (int ks = 0; ks < D / 16; ++ks)
+        tc5::mma_ss_if(leader, sd, a + uint64_t(((ks >> 2) * (BM * 128) + (ks & 3) * 32) >> 4),
+                       b + uint64_t(((ks >> 2) * (BN * 128) + (ks & 3) * 32) >> 4), id_qk, ks > 0);
       tc5::commit_if(leader, s_full(g, j & 1));
       __syncwarp();
       return true;
     };
-    // V tile, chunk-major: the head_dim halves of a chunk are box_rows * 128 B
-    // apart (LBO) and its two 8-key row groups 1 KB apart, or one block's box
-    // apart when a chunk spans two 8-row blocks (SBO).
-    const int box_rows = p.block_size < 16 ? p.block_size : 16;
-    const uint32_t v_lbo = box_rows * 128;
-    const uint32_t v_sbo = p.block_size >= 16 ? 1024u : uint32_t(D / 64) * 1024u;
     auto issue_pv = [&](int g, int j) -> bool {  // O_g += P(g, j) V_j, P from tensor memory
-      const int st = j % STAGES;
       // V landed with K: the scores of tile j, issued earlier, waited for both.
       if (!wait_all(p_full(g, j & 1), (j >> 1) & 1)) return false;
       tc5::fence_after();
-      const uint32_t vt = v_s + st * L::kKV;
+      const uint64_t b = dv + uint64_t((j % STAGES) * (L::kKV >> 4));
       const uint32_t pa = tmem + g * L::kColsPerGroup + (j & 1) * BN;
       const uint32_t od = tmem + g * L::kColsPerGroup + 2 * BN;
+      const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-      for (int ks = 0; ks < BN / 16; ++ks) {
-        const uint64_t db = tc5::sw128_desc(vt + ks * (32 * D), v_lbo, v_sbo);
-        tc5::mma_ts_if(leader, od, pa + ks * 8, db, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
-      }
+      for (int ks = 0; ks < BN / 16; ++ks)
+        tc5::mma_ts_if(leader, od, pa + ks * 8, b + uint64_t((ks * (32 * D)) >> 4), id_pv, ks > 0 ? 1u : acc0);
       tc5::commit_if(leader, pv_done(g, j & 1));
       __syncwarp();
       return true;
@@ -347,16 +358,16 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 1)
     if (ok) tc5::fence_after();
     for (int j = 0; j < 2 && ok; ++j)
       for (int g = 0; g < NWG && ok; ++g)
-        if (j < g_tiles(g)) ok = issue_qk(g, j);
+        if (j < gt(g)) ok = issue_qk(g, j);
     for (int j = 0; ok && j < ntiles; ++j) {
-      // On the CTA's last tile the group that zeroes the unused V rows goes first.
+      // On the CTA's last tile the query tile that zeroes the unused V rows goes first.
       const bool last = j == ntiles - 1;
-      for (int gi = 0; gi < NWG && ok; ++gi) {
+#pragma unroll
+      for (int gi = 0; gi < NWG; ++gi) {
         const int g = last ? NWG - 1 - gi : gi;
-        const bool uses = j < g_tiles(g);
-        if (uses) ok = issue_pv(g, j);
+        if (ok && j < gt(g)) ok = issue_pv(g, j);
         if (ok && gi == NWG - 1) tc5::commit_if(leader, &kv_empty[j % STAGES]);  // every P.V of tile j issued
-        if (ok && uses && j + 2 < g_tiles(g)) ok = issue_qk(g, j + 2);
+        if (ok && j + 2 < gt(g)) ok = issue_qk(g, j + 2);
       }
     }
     if (!ok && leader) set_err(p.err_flags, PA_ERRF_TIMEOUT);
