@@ -47,22 +47,43 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 
 # DRAM traffic of one decode-kernel launch (dram__bytes_read.sum +
-# dram__bytes_write.sum from one ncu --set full capture), keyed by workload;
-# reported only while the decode kernel's device sources hash to `src`.
+# dram__bytes_write.sum from one ncu capture: --set full, or those two
+# metrics alone), keyed by workload; reported only while the decode kernel's
+# device sources hash to `src`.
 NCU_TRAFFIC = {
     "llama7b-mha": {"bytes": 584_968_192 + 4_760_832, "src": "9d50e08d9a07cbcc"},
     "llama3-8b-gqa": {"bytes": 1_148_160_000 + 4_431_616, "src": "9d50e08d9a07cbcc"},
     "long-context-shared-prefix": {"bytes": 1_007_514_000 + 4_556_544, "src": "9d50e08d9a07cbcc"},
+    "llama13b-mha-bs8": {"bytes": 671_290_112 + 5_451_776, "src": "9d50e08d9a07cbcc"},
+    "llama13b-mha-bs16": {"bytes": 671_293_184 + 3_115_008, "src": "9d50e08d9a07cbcc"},
+    "llama13b-mha-bs32": {"bytes": 671_276_544 + 3_104_256, "src": "9d50e08d9a07cbcc"},
+    "llama13b-mha-bs64": {"bytes": 671_275_008 + 3_103_232, "src": "9d50e08d9a07cbcc"},
+    "tiny-mha": {"bytes": 315_136 + 0, "src": "9d50e08d9a07cbcc"},
 }
+
+
+# The same for one launch of the tcgen05 prefill kernel (ncu --set full).
+PREFILL_NCU_TRAFFIC = {
+    "chunked": {"bytes": 167_832_320 + 45_532_928, "src": "ade5ff18156f9ea0"},
+}
+
+
+def _sources_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "paged_kv_cache_368_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def kernel_source_hash() -> str:
     """Hash of the decode kernel's device code (the kernel whose traffic is quoted)."""
-    h = hashlib.sha256()
-    for f in ("paged_decode_kernel.cuh", "paged_merge.cuh", "pa_device.cuh"):
-        with open(os.path.join(ROOT, "paged_kv_cache_368_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return h.hexdigest()[:16]
+    return _sources_hash(("paged_decode_kernel.cuh", "paged_merge.cuh", "pa_device.cuh"))
+
+
+def prefill_source_hash() -> str:
+    """Hash of the tcgen05 prefill kernel's device code."""
+    return _sources_hash(("paged_prefill_tc.cu", "tcgen05.cuh", "exp2_poly.cuh", "pa_device.cuh"))
 
 
 def describe(wl) -> str:
@@ -740,6 +761,9 @@ def run_prefill(args):
     except Exception:
         pass
     peak = float(peaks.get("bf16_tflops", 1590.0))
+    peak_source = ("MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)" if "bf16_tflops" in peaks
+                   else "fallback (1.59 PFLOP/s, earlier cuBLAS burst measurement on this pool)")
+    psrc = prefill_source_hash()
     results = []
     for name, S, H, KVH, D, dtype, qlen, prefix in (
             ("ops-transformer example: 1 x 32 heads x 8192 tokens, d 64, fp16", 1, 32, 32, 64, "f16", [8192], [0]),
@@ -791,12 +815,17 @@ def run_prefill(args):
                "kv_bytes_logical": wl.kv_bytes(), "flops": flops, "kernel": "tcgen05",
                "mma_sync_us": ms_mma * 1e3, "mma_sync_tflops": flops / (ms_mma * 1e-3) / 1e12,
                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                            "traffic": None, "traffic_note": "kernel changed since the committed ncu capture"}}
+                            "traffic": None, "kernel_src": psrc}}
+        tr = PREFILL_NCU_TRAFFIC.get("chunked" if name.startswith("chunked") else name)
+        if tr and tr["src"] == psrc:
+            res["roofline"]["traffic"] = tr["bytes"]
+        else:
+            res["roofline"]["traffic_note"] = "no ncu capture of this kernel version on this workload"
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = prefill_cpu_baseline(wl, q, qlen, ctx, H, KVH, D, dtype)
         results.append(res)
     line = {"metric": "pa_prefill causal attention TFLOP/s", "op": "prefill", "n_gpus": 1, "steps": K, "warmup": W,
-            "peak_tflops": peak, "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)",
+            "peak_tflops": peak, "peak_source": peak_source,
             "results": results}
     print(json.dumps(line), flush=True)
     return 0
