@@ -568,7 +568,9 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
 
   const int S = p.num_seqs, H = p.num_heads;
   const int64_t NC = (int64_t)p.num_kv_heads * prefix[S];
-  const int64_t c0 = run_begin(gw, NC, W), c1 = run_begin(gw + 1, NC, W);
+  RunSplit rs;
+  rs.init(NC, W);
+  const int64_t c0 = rs.begin(gw), c1 = rs.begin(gw + 1);
   const int n = static_cast<int>(c1 - c0);
 
   // The run's split parts.  Its first segment (containing the run's first
@@ -687,7 +689,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     __syncwarp();
     int last = 0;
     if (lane == 0) {
-      int* t = p.ws_tickets + warp_of_chunk(a, NC, W);
+      int* t = p.ws_tickets + rs.warp_of(a);
       int before;
       asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(before) : "l"(t), "r"(mine) : "memory");
       last = before + mine == u.nc;
@@ -698,7 +700,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     if (last) {
       merge_split_unit<T, D, G>(p.ws_ml, p.ws_o,
                                 static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D, a,
-                                u.nc, NC, W, lane);
+                                u.nc, rs, lane);
     }
     (first ? ticket_f : ticket_l) = true;
   };

@@ -13,21 +13,50 @@
 namespace pa {
 
 // The global chunk order is split evenly over W warps: warp w runs chunks
-// [floor(w*NC/W), floor((w+1)*NC/W)).
-__device__ __forceinline__ int64_t run_begin(int64_t w, int64_t NC, int W) { return w * NC / W; }
+// [floor(w*NC/W), floor((w+1)*NC/W)).  The run bounds are evaluated without
+// 64-bit division (a long emulated sequence that every merge and ticket
+// used to pay several times): with NC = q*W + r, floor(w*NC/W) =
+// w*q + floor(w*r/W), and w*r < W*W fits 32 bits.
+struct RunSplit {
+  int64_t NC;
+  int64_t q;  // NC / W
+  uint32_t r;  // NC % W
+  int W;
 
-// The warp whose run holds global chunk g: the w with
-// floor(w*NC/W) <= g < floor((w+1)*NC/W), i.e. ceil((g+1)*W/NC) - 1.
-__device__ __forceinline__ int warp_of_chunk(int64_t g, int64_t NC, int W) {
-  return static_cast<int>(((g + 1) * W + NC - 1) / NC - 1);
-}
+  __device__ __forceinline__ void init(int64_t nc, int w) {
+    NC = nc;
+    W = w;
+    q = nc / w;
+    r = static_cast<uint32_t>(nc - q * w);
+  }
 
-// Partial slot of warp w's part of the unit that starts at global chunk a:
-// slot 2w holds a warp's first segment, slot 2w+1 its last.  The part is the
-// warp's first segment exactly when its run starts at or after a.
-__device__ __forceinline__ int64_t partial_slot(int64_t w, int64_t a, int64_t NC, int W) {
-  return 2 * w + (run_begin(w, NC, W) >= a ? 0 : 1);
-}
+  __device__ __forceinline__ int64_t begin(int w) const {
+    return (int64_t)w * q + (int64_t)((static_cast<uint32_t>(w) * r) / static_cast<uint32_t>(W));
+  }
+
+  // The warp whose run holds global chunk g: the w with begin(w) <= g <
+  // begin(w+1), which is ceil((g+1)*W/NC) - 1.  That quotient (below 2^11)
+  // is estimated in single precision, whose few roundings move it by far
+  // less than 1, so the estimate is off by at most one; the run bounds then
+  // settle it exactly.
+  __device__ __forceinline__ int warp_of(int64_t g) const {
+    if (NC <= 0) return 0;
+    const float x = static_cast<float>(g + 1) * static_cast<float>(W) / static_cast<float>(NC);
+    int w = static_cast<int>(ceilf(x)) - 1;
+    w = w < 0 ? 0 : (w > W - 1 ? W - 1 : w);
+    if (begin(w) > g) {
+      --w;
+    } else if (w + 1 < W && begin(w + 1) <= g) {
+      ++w;
+    }
+    return w;
+  }
+
+  // Partial slot of warp w's part of the unit that starts at global chunk a:
+  // slot 2w holds a warp's first segment, slot 2w+1 its last.  The part is
+  // the warp's first segment exactly when its run starts at or after a.
+  __device__ __forceinline__ int partial_slot(int w, int64_t a) const { return 2 * w + (begin(w) >= a ? 0 : 1); }
+};
 
 // Merge the partials of the unit of `nc` chunks starting at global chunk `a`
 // and write its G q-head rows (out_row -> [G][D]).  One warp, two phases per
@@ -47,14 +76,14 @@ __device__ __forceinline__ int64_t partial_slot(int64_t w, int64_t a, int64_t NC
 // skipped) has weight 0.
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_split_unit(const float2* ws_ml, const float* ws_o, T* out_row, int64_t a,
-                                                 int nc, int64_t NC, int W, int lane) {
+                                                 int nc, const RunSplit& rs, int lane) {
   using E = Elem<T>;
   constexpr int kItems = G * D / 4;          // float4 outputs
   constexpr int kPerLane = (kItems + 31) / 32;
   constexpr int kBatch = kPerLane >= 8 ? 1 : 4;  // contributors in flight in phase 2
   constexpr int kHeadItems = D / 4;          // float4 columns of one q-head
-  const int w0 = warp_of_chunk(a, NC, W);
-  const int nw = warp_of_chunk(a + nc - 1, NC, W) - w0 + 1;
+  const int w0 = rs.warp_of(a);
+  const int nw = rs.warp_of(a + nc - 1) - w0 + 1;
   float M[G], L[G];  // running maximum (log2 units) and weighted sum of l, per q-head
   float4 acc[kPerLane];
 #pragma unroll
@@ -69,8 +98,8 @@ __device__ __forceinline__ void merge_split_unit(const float2* ws_ml, const floa
     // ---- phase 1: this lane's contributor of the block
     const int wj = w0 + base + lane;
     // Warps with an empty run (more warps than chunks) wrote nothing.
-    const bool has = base + lane < nw && run_begin(wj, NC, W) < run_begin(wj + 1, NC, W);
-    const int slot = has ? static_cast<int>(partial_slot(wj, a, NC, W)) : 0;
+    const bool has = base + lane < nw && rs.begin(wj) < rs.begin(wj + 1);
+    const int slot = has ? rs.partial_slot(wj, a) : 0;
     float wgt[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
