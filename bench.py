@@ -51,14 +51,14 @@ L2_BYTES = 126 * 1024 * 1024
 # metrics alone), keyed by workload; reported only while the decode kernel's
 # device sources hash to `src`.
 NCU_TRAFFIC = {
-    "llama7b-mha": {"bytes": 584_968_192 + 4_760_832, "src": "9d50e08d9a07cbcc"},
-    "llama3-8b-gqa": {"bytes": 1_148_160_000 + 4_431_616, "src": "9d50e08d9a07cbcc"},
-    "long-context-shared-prefix": {"bytes": 1_007_514_000 + 4_556_544, "src": "9d50e08d9a07cbcc"},
-    "llama13b-mha-bs8": {"bytes": 671_290_112 + 5_451_776, "src": "9d50e08d9a07cbcc"},
-    "llama13b-mha-bs16": {"bytes": 671_293_184 + 3_115_008, "src": "9d50e08d9a07cbcc"},
-    "llama13b-mha-bs32": {"bytes": 671_276_544 + 3_104_256, "src": "9d50e08d9a07cbcc"},
-    "llama13b-mha-bs64": {"bytes": 671_275_008 + 3_103_232, "src": "9d50e08d9a07cbcc"},
-    "tiny-mha": {"bytes": 315_136 + 0, "src": "9d50e08d9a07cbcc"},
+    "llama7b-mha": {"bytes": 584_962_816 + 3_268_096, "src": "0fc3b1941294cf11"},
+    "llama3-8b-gqa": {"bytes": 1_148_157_696 + 3_682_304, "src": "0fc3b1941294cf11"},
+    "long-context-shared-prefix": {"bytes": 1_006_903_040 + 3_442_176, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs8": {"bytes": 671_289_088 + 2_937_344, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs16": {"bytes": 671_280_128 + 3_345_920, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs32": {"bytes": 671_282_688 + 3_188_480, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs64": {"bytes": 671_275_264 + 3_356_416, "src": "0fc3b1941294cf11"},
+    "tiny-mha": {"bytes": 315_392 + 0, "src": "0fc3b1941294cf11"},
 }
 
 
