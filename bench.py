@@ -45,6 +45,8 @@ UNIT = "GB/s"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
+PREFILL_BURST_S = 0.02  # device time of the burst figure (against the burst bf16 peak)
+PREFILL_SUSTAINED_S = 1.0  # device time of the sustained figure (against the sustained peak)
 
 # DRAM traffic of one decode-kernel launch (dram__bytes_read.sum +
 # dram__bytes_write.sum from one ncu capture: --set full, or those two
@@ -763,6 +765,10 @@ def run_prefill(args):
     peak = float(peaks.get("bf16_tflops", 1590.0))
     peak_source = ("MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)" if "bf16_tflops" in peaks
                    else "fallback (1.59 PFLOP/s, earlier cuBLAS burst measurement on this pool)")
+    peak_sus = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    peak_sus_source = ("MEASURED_PEAKS.json bf16_tflops_sustained (cuBLAS, seconds under the power cap)"
+                       if "bf16_tflops_sustained" in peaks
+                       else "fallback (~1.4 PFLOP/s, cuBLAS sustained under the power cap on this pool)")
     psrc = prefill_source_hash()
     results = []
     for name, S, H, KVH, D, dtype, qlen, prefix in (
@@ -791,20 +797,32 @@ def run_prefill(args):
             libpaged.prefill(out, q, cu, kc, vc, tables, ctx_t, float(wl.scale), max_q_len=max(qlen),
                              max_context_len=max(ctx), legacy_mma=legacy)
 
-        def timed(legacy):
+        def timed(legacy, seconds):
+            """ms per call over at most K calls and about `seconds` of device
+            time.  Seconds of back-to-back tensor work bring the power cap's
+            lower clocks, so a short burst is set against the burst peak and a
+            long run against the sustained one."""
             for _ in range(W):
                 call(legacy)
             torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            for _ in range(K):
+            call(legacy)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            n = max(1, min(K, int(seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+            e0.record()
+            for _ in range(n):
                 call(legacy)
             e1.record()
             torch.cuda.synchronize(dev)
-            return e0.elapsed_time(e1) / K
+            calls[(legacy, seconds)] = n
+            return e0.elapsed_time(e1) / n
 
-        ms = timed(False)
-        ms_mma = timed(True)
+        calls = {}
+        ms = timed(False, PREFILL_BURST_S)
+        ms_mma = timed(True, PREFILL_BURST_S)
+        ms_sus = timed(False, PREFILL_SUSTAINED_S)
         # causal FLOPs: row at position p does 2 * 2 * D * (p + 1) per q-head (QK and PV)
         flops = 0
         for n, c in zip(qlen, ctx):
@@ -814,6 +832,10 @@ def run_prefill(args):
         res = {"workload": name, "us": ms * 1e3, "tflops": tf, "frac_of_bf16_peak": tf / peak,
                "kv_bytes_logical": wl.kv_bytes(), "flops": flops, "kernel": "tcgen05",
                "mma_sync_us": ms_mma * 1e3, "mma_sync_tflops": flops / (ms_mma * 1e-3) / 1e12,
+               "timed_calls": calls[(False, PREFILL_BURST_S)], "mma_sync_timed_calls": calls[(True, PREFILL_BURST_S)],
+               "sustained": {"us": ms_sus * 1e3, "tflops": flops / (ms_sus * 1e-3) / 1e12,
+                             "calls": calls[(False, PREFILL_SUSTAINED_S)], "peak": peak_sus,
+                             "frac": flops / (ms_sus * 1e-3) / 1e12 / peak_sus, "peak_source": peak_sus_source},
                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                             "traffic": None, "kernel_src": psrc}}
         tr = PREFILL_NCU_TRAFFIC.get("chunked" if name.startswith("chunked") else name)
