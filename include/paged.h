@@ -124,11 +124,12 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_h
  *   (fewer, longer per-warp runs -> fewer split partitions).  The result is
  *   the same attention for every choice, up to fp32 rounding order.
  * Supported: head_dim in {64, 128}; block_size in {8, 16, 32, 64};
- *   num_heads/num_kv_heads in {1, 2, 4, 8}; 1 <= num_seqs <= 16384 while
- *   the per-sequence prefix table (4 bytes a sequence) fits in shared memory
- *   beside the pipeline stages (PA_ERR_UNSUPPORTED otherwise);
- *   num_kv_heads < 32768;
- *   num_seqs * num_kv_heads * ceil(max_context_len/16) < 2^31.
+ *   num_heads/num_kv_heads in {1, 2, 4, 8}; num_kv_heads < 32768.  One
+ *   launch takes at most 16384 sequences (its per-sequence prefix table, 4
+ *   bytes a sequence, lives in shared memory); a larger batch runs as
+ *   several launches of up to 16384 sequences, in order on `stream`, sharing
+ *   the workspace.  Per launch, sequences * num_kv_heads *
+ *   ceil(max_context_len/16) < 2^31 (PA_ERR_UNSUPPORTED otherwise).
  */
 PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,

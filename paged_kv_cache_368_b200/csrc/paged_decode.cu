@@ -179,9 +179,13 @@ pa_status plan_decode(int num_seqs, int max_blocks_per_seq, int max_context_len,
   if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (!valid_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-  if (num_seqs > kMaxSeqs || num_kv_heads >= (1 << 15)) return PA_ERR_UNSUPPORTED;
+  if (num_kv_heads >= (1 << 15)) return PA_ERR_UNSUPPORTED;
+  // One launch takes at most kMaxSeqs sequences (its per-sequence prefix
+  // table lives in shared memory); pa_decode runs a larger batch as several
+  // launches, so the limits below are those of one launch.
+  const int64_t batch = std::min(num_seqs, kMaxSeqs);
   const int64_t cap64 = std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * block_size);
-  const int64_t upper = (int64_t)num_seqs * num_kv_heads * ((cap64 + kChunk - 1) / kChunk);
+  const int64_t upper = batch * num_kv_heads * ((cap64 + kChunk - 1) / kChunk);
   if (upper >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   if (num_blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
   plan->G = G;
@@ -258,32 +262,57 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
 
   pa::DecodeParams p;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.out = out;
-  p.q = q;
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
-  p.ws_tickets = reinterpret_cast<int*>(ws + L.tickets);
-  p.ws_ml = reinterpret_cast<float2*>(ws + L.ml);
-  p.ws_o = reinterpret_cast<float*>(ws + L.o);
   p.err_flags = err_flags;
   p.num_blocks = num_blocks;
-  p.num_seqs = num_seqs;
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.ctx_cap = plan.ctx_cap;
   p.max_context_len = max_context_len;
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;
   p.block_size = block_size;
-  p.total_warps = ctas * warps;
   p.scale_log2 = scale * 1.4426950408889634f;
 
+  // Batches of at most kMaxSeqs sequences, one launch each, in order on
+  // `stream`.  They share the workspace: a launch touches it only after its
+  // programmatic wait for the previous one, and leaves the ticket counters at
+  // zero.  The first batch is the largest, so its grid and layout (checked
+  // above) bound every later one's.
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == PA_F16) {
-    return head_dim == 128 ? dispatch_g<__half, 128>(G, km, vm, p, ctas, s, dev)
-                           : dispatch_g<__half, 64>(G, km, vm, p, ctas, s, dev);
+  const size_t row_bytes = (size_t)num_heads * head_dim * 2;  // one sequence of q or out
+  for (int s0 = 0; s0 < num_seqs; s0 += pa::kMaxSeqs) {
+    const int nb = std::min(pa::kMaxSeqs, num_seqs - s0);
+    int bctas = ctas;
+    pa::WsLayout BL = L;
+    if (s0 > 0) {  // the last batch may be smaller: its own grid
+      pa::DecodePlan bp;
+      const pa_status bst = pa::plan_decode(nb, max_blocks_per_seq, max_context_len, scale, num_heads, num_kv_heads,
+                                            head_dim, block_size, num_blocks, dtype, max_ctas, &bp);
+      if (bst != PA_OK) return bst;
+      const pa_status bgst = pa::plan_decode_grid(max_ctas, &bp);
+      if (bgst != PA_OK) return bgst;
+      bctas = bp.ctas;
+      BL = bp.layout;
+    }
+    p.out = static_cast<uint8_t*>(out) + (size_t)s0 * row_bytes;
+    p.q = static_cast<const uint8_t*>(q) + (size_t)s0 * row_bytes;
+    p.block_tables = block_tables + (size_t)s0 * max_blocks_per_seq;
+    p.context_lens = context_lens + s0;
+    p.num_seqs = nb;
+    p.ws_tickets = reinterpret_cast<int*>(ws + BL.tickets);
+    p.ws_ml = reinterpret_cast<float2*>(ws + BL.ml);
+    p.ws_o = reinterpret_cast<float*>(ws + BL.o);
+    p.total_warps = bctas * warps;
+    pa_status lst;
+    if (dtype == PA_F16) {
+      lst = head_dim == 128 ? dispatch_g<__half, 128>(G, km, vm, p, bctas, s, dev)
+                            : dispatch_g<__half, 64>(G, km, vm, p, bctas, s, dev);
+    } else {
+      lst = head_dim == 128 ? dispatch_g<__nv_bfloat16, 128>(G, km, vm, p, bctas, s, dev)
+                            : dispatch_g<__nv_bfloat16, 64>(G, km, vm, p, bctas, s, dev);
+    }
+    if (lst != PA_OK) return lst;
   }
-  return head_dim == 128 ? dispatch_g<__nv_bfloat16, 128>(G, km, vm, p, ctas, s, dev)
-                         : dispatch_g<__nv_bfloat16, 64>(G, km, vm, p, ctas, s, dev);
+  return PA_OK;
 }
 
 extern "C" const char* pa_status_string(pa_status status) {

@@ -63,7 +63,9 @@ def test_decode_host_checks(lib):
     assert _decode(lib, H=48, KVH=3) == U  # group of 16 q-heads
     assert _decode(lib, D=96) == U
     assert _decode(lib, BS=24) == U
-    assert _decode(lib, S=16385) == U  # above the sequence limit
+    # one launch's chunk count: 16384 sequences x 4096 kv-heads x 32 chunks = 2^31
+    assert _decode(lib, S=16384, H=4096, KVH=4096, mb=32, maxctx=512) == U
+    assert _decode(lib, S=16385, H=4096, KVH=4096, mb=32, maxctx=512) == U  # the same per launch
     assert _decode(lib, KVH=1 << 15, H=1 << 15) == U
     assert _decode(lib, out=None) == I
     assert _decode(lib, q=24) == I  # misaligned
@@ -92,7 +94,7 @@ def test_decode_static_host_checks(lib):
     assert _decode_static(lib, D=80) == U
     assert _decode_static(lib, BS=128) == U
     assert _decode_static(lib, H=64, KVH=4) == U  # group of 16
-    assert _decode_static(lib, S=20000) == U
+    assert _decode_static(lib, S=20000, H=4096, KVH=4096, mb=32, maxctx=512) == U  # 2^31 chunks in a launch
     assert _decode_static(lib, S=0) == libpaged.PA_OK
 
 
