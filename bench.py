@@ -53,14 +53,14 @@ PREFILL_SUSTAINED_S = 1.0  # device time of the sustained figure (against the su
 # metrics alone), keyed by workload; reported only while the decode kernel's
 # device sources hash to `src`.
 NCU_TRAFFIC = {
-    "llama7b-mha": {"bytes": 584_982_528 + 3_243_264, "src": "d2ea5ac9ce3f3358"},
-    "llama3-8b-gqa": {"bytes": 1_148_191_232 + 4_022_016, "src": "d2ea5ac9ce3f3358"},
-    "long-context-shared-prefix": {"bytes": 1_007_351_296 + 3_378_944, "src": "d2ea5ac9ce3f3358"},
-    "llama13b-mha-bs8": {"bytes": 671_373_056 + 3_247_616, "src": "d2ea5ac9ce3f3358"},
-    "llama13b-mha-bs16": {"bytes": 671_294_720 + 3_350_528, "src": "d2ea5ac9ce3f3358"},
-    "llama13b-mha-bs32": {"bytes": 671_295_488 + 3_205_632, "src": "d2ea5ac9ce3f3358"},
-    "llama13b-mha-bs64": {"bytes": 671_293_952 + 4_097_024, "src": "d2ea5ac9ce3f3358"},
-    "tiny-mha": {"bytes": 314_880 + 0, "src": "d2ea5ac9ce3f3358"},
+    "llama7b-mha": {"bytes": 584_962_816 + 3_268_096, "src": "0fc3b1941294cf11"},
+    "llama3-8b-gqa": {"bytes": 1_148_157_696 + 3_682_304, "src": "0fc3b1941294cf11"},
+    "long-context-shared-prefix": {"bytes": 1_006_903_040 + 3_442_176, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs8": {"bytes": 671_289_088 + 2_937_344, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs16": {"bytes": 671_280_128 + 3_345_920, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs32": {"bytes": 671_282_688 + 3_188_480, "src": "0fc3b1941294cf11"},
+    "llama13b-mha-bs64": {"bytes": 671_275_264 + 3_356_416, "src": "0fc3b1941294cf11"},
+    "tiny-mha": {"bytes": 315_392 + 0, "src": "0fc3b1941294cf11"},
 }
 
 

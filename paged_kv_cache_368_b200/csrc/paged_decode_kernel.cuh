@@ -11,7 +11,6 @@ namespace pa {
 
 constexpr int kChunk = 16;       // tokens per pipeline stage
 constexpr int kMaxSeqs = 16384;  // prefix table lives in shared memory (4 bytes a sequence)
-constexpr int kDeferMinChunks = 8;  // run chunks still to stream for a split unit's merge to wait for them
 #ifndef PA_CORE_WARPS
 #define PA_CORE_WARPS 8
 #endif
@@ -676,11 +675,7 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
   // whose addition completes the unit's count merges every part and writes
   // the output, so no warp ever waits for another.
   bool ticket_f = false, ticket_l = false;
-  using PM = PrefetchedMerge<T, D, G>;
-  PM pm_f, pm_l;  // merges whose loads are in flight, one per split segment
-  pm_f.clear();
-  pm_l.clear();
-  auto take_ticket = [&](bool first, bool defer) {
+  auto take_ticket = [&](bool first) {
     const int64_t a = first ? af : al;
     const UnitPos& u = first ? uf : ul;
     const int mine = first ? mine_f : mine_l;
@@ -703,14 +698,9 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
     last = __shfl_sync(kFull, last, 0);
     __syncwarp();
     if (last) {
-      T* out_row = static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D;
-      // Small units on the CUDA-core path: loads now, weighted sum once the
-      // run has been streamed.
-      bool deferred = false;
-      if constexpr (PM::kApplies) {
-        if (defer) deferred = (first ? pm_f : pm_l).start(p.ws_ml, p.ws_o, out_row, a, u.nc, rs, lane);
-      }
-      if (!deferred) merge_split_unit<T, D, G>(p.ws_ml, p.ws_o, out_row, a, u.nc, rs, lane);
+      merge_split_unit<T, D, G>(p.ws_ml, p.ws_o,
+                                static_cast<T*>(p.out) + ((int64_t)u.seq * H + (int64_t)u.head * G) * D, a,
+                                u.nc, rs, lane);
     }
     (first ? ticket_f : ticket_l) = true;
   };
@@ -775,14 +765,9 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
       } else {
         const int slot = 2 * gw + (seg_has_run_start ? 0 : 1);
         st.write_partial(p.ws_o + (int64_t)slot * G * D, p.ws_ml + (int64_t)slot * G, lane);
-        // defer the merge only when enough of the run is left to hide its loads
-        take_ticket(seg_has_run_start, n - 1 - k >= kDeferMinChunks);
+        take_ticket(seg_has_run_start);
       }
     }
-  }
-  if constexpr (PM::kApplies) {
-    if (pm_f.active) pm_f.finish(lane);
-    if (pm_l.active) pm_l.finish(lane);
   }
   if (timed_out) {
     set_err(p.err_flags, PA_ERRF_TIMEOUT);
@@ -791,8 +776,8 @@ __global__ void __launch_bounds__(Shape<D, G>::kWarps * 32, 1)
       mbar_wait_bounded(&bars[warp * DEPTH + (kk % DEPTH)], (kk / DEPTH) & 1, kWaitLimitNs);
     // The split parts not reached still count their chunks, so the counters
     // return to zero (their outputs are flagged as not written).
-    if (part_f && !ticket_f) take_ticket(true, false);
-    if (part_l && !ticket_l) take_ticket(false, false);
+    if (part_f && !ticket_f) take_ticket(true);
+    if (part_l && !ticket_l) take_ticket(false);
   }
 }
 

@@ -183,102 +183,4 @@ __device__ __forceinline__ void merge_split_unit(const float2* ws_ml, const floa
   }
 }
 
-// The same merge for a unit of at most kParts parts whose G*D/4 float4
-// outputs fit one per lane (G = 1 at head_dim 128; G <= 2 at head_dim 64),
-// in two halves.  start() issues every load at once, right after the ticket:
-// lane j the (m, l) of contributor j, each lane its float4 column of every
-// contributor's o.  finish() forms the weights and the weighted sum, and is
-// called once the warp has streamed the rest of its run.  Under the TMA
-// stream of a whole SM, global loads through the LSU wait a long time (the
-// merge's loads were most of its cost, and issuing them one chunk ahead hid
-// none of it); the split parts come first in a run on this path, so the loads
-// have the whole run to land.  The arithmetic and its order are those of
-// merge_split_unit, so both give the same bits.
-template <typename T, int D, int G>
-struct PrefetchedMerge {
-  static constexpr int kParts = 4;
-  static constexpr int kItems = G * D / 4;  // float4 outputs
-  static constexpr bool kApplies = kItems <= 32;
-  static constexpr int kHeadItems = D / 4;
-  float2 ml[G];
-  float4 o[kParts];
-  T* out_row;
-  int nw;
-  bool active;
-
-  __device__ __forceinline__ void clear() { active = false; }
-
-  // Issue the loads of the unit of `nc` chunks starting at global chunk `a`;
-  // false (nothing issued) when the unit has more than kParts parts.
-  __device__ __forceinline__ bool start(const float2* ws_ml, const float* ws_o, T* out, int64_t a, int nc,
-                                        const RunSplit& rs, int lane) {
-    const int w0 = rs.warp_of(a);
-    const int parts = rs.warp_of(a + nc - 1) - w0 + 1;
-    if (parts > kParts) return false;
-    const int wj = w0 + lane;
-    const bool has = lane < parts && rs.begin(wj) < rs.begin(wj + 1);
-    const int slot = has ? rs.partial_slot(wj, a) : 0;
-#pragma unroll
-    for (int g = 0; g < G; ++g) ml[g] = has ? __ldcg(ws_ml + (int64_t)slot * G + g) : make_float2(-INFINITY, 0.f);
-    const int g = lane / kHeadItems, d4 = lane % kHeadItems;
-#pragma unroll
-    for (int j = 0; j < kParts; ++j) {
-      const bool use = j < parts && __shfl_sync(kFull, has, j);
-      const int sl = __shfl_sync(kFull, slot, j);
-      o[j] = (use && lane < kItems) ? __ldcg(reinterpret_cast<const float4*>(ws_o + ((int64_t)sl * G + g) * D) + d4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    out_row = out;
-    nw = parts;
-    active = true;
-    return true;
-  }
-
-  __device__ __forceinline__ void finish(int lane) {
-    using E = Elem<T>;
-    float wgt[G], L[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float mb = ml[g].x;
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
-      wgt[g] = ml[g].x == -INFINITY ? 0.f : fast_exp2(ml[g].x - mb);
-      float ls = wgt[g] * ml[g].y;
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) ls += __shfl_xor_sync(kFull, ls, off);
-      L[g] = ls;
-    }
-    const int gi = lane / kHeadItems, d4 = lane % kHeadItems;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < kParts; ++j) {
-      float w = 0.f;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float wj = __shfl_sync(kFull, wgt[g], j);
-        w = g == gi ? wj : w;
-      }
-      w = j < nw ? w : 0.f;
-      // a part of weight 0 adds 0 * 0, as in merge_split_unit (which does not
-      // load it): whatever its o holds cannot reach the output
-      const float4 oj = w != 0.f ? o[j] : make_float4(0.f, 0.f, 0.f, 0.f);
-      acc.x = fmaf(w, oj.x, acc.x);
-      acc.y = fmaf(w, oj.y, acc.y);
-      acc.z = fmaf(w, oj.z, acc.z);
-      acc.w = fmaf(w, oj.w, acc.w);
-    }
-    if (lane < kItems) {
-      float lg = 0.f;
-#pragma unroll
-      for (int g = 0; g < G; ++g) lg = g == gi ? L[g] : lg;
-      const float inv = lg > 0.f ? 1.f / lg : 0.f;
-      uint2 u;
-      u.x = E::pack(acc.x * inv, acc.y * inv);
-      u.y = E::pack(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(out_row + gi * D + d4 * 4) = u;
-    }
-    active = false;
-  }
-};
-
 }  // namespace pa
