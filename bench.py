@@ -67,6 +67,7 @@ NCU_TRAFFIC = {
 # The same for one launch of the tcgen05 prefill kernel (ncu --set full).
 PREFILL_NCU_TRAFFIC = {
     "chunked": {"bytes": 167_832_320 + 45_532_928, "src": "ade5ff18156f9ea0"},
+    "d64": {"bytes": 100_769_280 + 16_449_280, "src": "ade5ff18156f9ea0"},
 }
 
 
@@ -853,7 +854,7 @@ def run_prefill(args):
                              "frac": flops / (ms_sus * 1e-3) / 1e12 / peak_sus, "peak_source": peak_sus_source},
                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                             "traffic": None, "kernel_src": psrc}}
-        tr = PREFILL_NCU_TRAFFIC.get("chunked" if name.startswith("chunked") else name)
+        tr = PREFILL_NCU_TRAFFIC.get("chunked" if name.startswith("chunked") else "d64")
         if tr and tr["src"] == psrc:
             res["roofline"]["traffic"] = tr["bytes"]
         else:
